@@ -1,0 +1,135 @@
+"""Python binding of the fp8lite C ABI (include/fp8lite.h).
+
+Argument marshalling only: every step of quantization and of the GEMM runs in
+the CUDA library ``libfp8lite.so`` built in this package directory. The
+functions carry the C names and argument order; buffers may be given as
+torch tensors (their ``data_ptr()`` is passed) or as integer device
+addresses, and ``stream`` defaults to torch's current CUDA stream. A non-OK
+status raises ``Fp8Error``. Importing fails loudly when the library has not
+been built: there is no fallback path.
+"""
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfp8lite.so")
+
+FP8_E4M3, FP8_E5M2 = 0, 1
+FP8_NT, FP8_NN, FP8_TN = 0, 1, 2
+FP8_OK = 0
+FP8_ERR_INVALID_ARG = 1
+FP8_ERR_ALIGNMENT = 2
+FP8_ERR_UNSUPPORTED = 3
+FP8_ERR_CUDA = 4
+FP8_ERR_DEVICE_TIMEOUT = 5
+FP8_RING_HISTORY = 16
+FP8_RING_BYTES = 80
+
+
+class Fp8Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+class fp8_ring(ctypes.Structure):
+    """Host image of the device ring (80 bytes)."""
+    _fields_ = [("hist", ctypes.c_float * FP8_RING_HISTORY), ("scale", ctypes.c_float),
+                ("idx", ctypes.c_uint32), ("amax_bits", ctypes.c_uint32), ("ticket", ctypes.c_uint32)]
+
+
+assert ctypes.sizeof(fp8_ring) == FP8_RING_BYTES
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python -m fp8_delayed_scaling_quantize_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I64, I, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+    sig = {
+        "fp8_status_string": (ctypes.c_char_p, [I]),
+        "fp8_abi_version": (I, []),
+        "fp8_ring_init": (I, [P, F, P]),
+        "fp8_ring_get": (I, [P, P, P]),
+        "fp8_ring_set": (I, [P, P, P]),
+        "fp8_quantize": (I, [P, I64, I, P, P, P, P, P]),
+        "fp8_mm": (I, [P, I, P, I, P, P, I, I64, I64, I64, I64, I64, I64, I64, P, P, I, P, P]),
+        "fp8_last_device_error": (I, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x or None
+    return x.data_ptr() or None
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    if isinstance(stream, int):
+        return stream or None
+    return stream.cuda_stream or None
+
+
+def _check(status: int, where: str) -> int:
+    if status != FP8_OK:
+        raise Fp8Error(status, where)
+    return status
+
+
+def status_string(status: int) -> str:
+    return lib.fp8_status_string(int(status)).decode()
+
+
+def fp8_abi_version() -> int:
+    return lib.fp8_abi_version()
+
+
+def fp8_ring_init(ring, init_scale: float = 1.0, stream=None):
+    return _check(lib.fp8_ring_init(_ptr(ring), float(init_scale), _stream(stream)), "fp8_ring_init")
+
+
+def fp8_ring_get(ring, stream=None) -> fp8_ring:
+    host = fp8_ring()
+    _check(lib.fp8_ring_get(_ptr(ring), ctypes.byref(host), _stream(stream)), "fp8_ring_get")
+    return host
+
+
+def fp8_ring_set(ring, host: fp8_ring, stream=None):
+    return _check(lib.fp8_ring_set(_ptr(ring), ctypes.byref(host), _stream(stream)), "fp8_ring_set")
+
+
+def fp8_quantize(x, n, fmt, ring, out8, amax_out, scale_out, stream=None):
+    return _check(lib.fp8_quantize(_ptr(x), int(n), int(fmt), _ptr(ring), _ptr(out8), _ptr(amax_out),
+                                   _ptr(scale_out), _stream(stream)), "fp8_quantize")
+
+
+def fp8_mm(a8, fa, b8, fb, sa, sb, layout, M, N, K, batch, stride_a, stride_b, stride_c, bias,
+           bias_scale, bias_fmt, out, stream=None):
+    return _check(lib.fp8_mm(_ptr(a8), int(fa), _ptr(b8), int(fb), _ptr(sa), _ptr(sb), int(layout),
+                             int(M), int(N), int(K), int(batch), int(stride_a), int(stride_b),
+                             int(stride_c), _ptr(bias), _ptr(bias_scale), int(bias_fmt), _ptr(out),
+                             _stream(stream)), "fp8_mm")
+
+
+def fp8_last_device_error():
+    return _check(lib.fp8_last_device_error(), "fp8_last_device_error")
+
+
+def raw_status(fn_name: str, *args) -> int:
+    """Call a C entry point with pre-marshalled arguments and return its
+    status without raising (used to test argument validation)."""
+    return getattr(lib, fn_name)(*args)

@@ -1,0 +1,281 @@
+// Per-tensor FP8 quantization with amax reduction and the delayed-scaling
+// ring finalized on the device (sm_100a).
+//
+// Method: AstrAI commit log astrai/extension/fp8.py @4dc5e923 -- the amax is
+// taken over the unquantized input (bullets on the amax bug), and the quantize
+// kernel's last thread block (threadfence + counter election) folds the amax
+// into hist[idx], reduces the window and publishes the next scale with no
+// extra launch (bullet on the last-block epilogue). The scale used by the call
+// is returned separately because the finalize replaces the ring's scale
+// (astrai/extension/fp8.py @f4c44ebf, bullet on the scale snapshot).
+//
+// Kernel design (HBM-bound, 3 bytes per element when delayed):
+//  * each thread moves 8 bf16 (one 16-byte load) -> 8 codes (one 8-byte
+//    store); a warp's load instruction covers 512 contiguous bytes and its
+//    store 256 contiguous bytes; four such units are in flight per thread;
+//  * x * s is one fp32 multiply (round-to-nearest, no flush-to-zero), then
+//    the hardware pair conversion cvt.rn.satfinite.{e4m3x2,e5m2x2}.f32 does
+//    the nearest-even FP8 rounding with saturation -- never through fp16;
+//  * amax: fmaxf per thread (NaN is ignored), then warp redux.sync max on the
+//    bit patterns (non-negative floats order like unsigned integers), a
+//    shared-memory pass over the block's warps and one atomicMax per block;
+//  * delayed: one launch; the block that draws the last ticket finalizes the
+//    ring and resets its accumulator and ticket, so the ring is ready for the
+//    next call (and for CUDA-graph replay) with no host involvement;
+//  * current: memset of the caller's amax word, an amax-only pass, then the
+//    quantize pass that derives the scale from that amax. For tensors that
+//    fit in L2 the second read is served from L2.
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace fp8lite {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kUnroll = 4;  // 16-byte units in flight per thread
+
+enum Mode { kDelayed = 0, kCurrentQuant = 1, kAmaxOnly = 2 };
+
+template <int FMT>
+__device__ __forceinline__ uint32_t cvt_pair(float lo, float hi) {
+    // The first source lands in the upper byte, the second in the lower one.
+    uint16_t r;
+    if (FMT == FP8_E4M3) {
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    } else {
+        asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    }
+    return r;
+}
+
+// bf16 is the upper half of an fp32: widening is a bit shift, exact for
+// every value including subnormals.
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+template <int FMT>
+__device__ __forceinline__ uint32_t quant4(uint32_t w0, uint32_t w1, float s, float& m) {
+    const float a = bf_lo(w0), b = bf_hi(w0), c = bf_lo(w1), d = bf_hi(w1);
+    m = fmaxf(m, fabsf(a));
+    m = fmaxf(m, fabsf(b));
+    m = fmaxf(m, fabsf(c));
+    m = fmaxf(m, fabsf(d));
+    const uint32_t lo = cvt_pair<FMT>(__fmul_rn(a, s), __fmul_rn(b, s));
+    const uint32_t hi = cvt_pair<FMT>(__fmul_rn(c, s), __fmul_rn(d, s));
+    return lo | (hi << 16);
+}
+
+__device__ __forceinline__ void amax4(uint32_t w0, uint32_t w1, float& m) {
+    m = fmaxf(m, fabsf(bf_lo(w0)));
+    m = fmaxf(m, fabsf(bf_hi(w0)));
+    m = fmaxf(m, fabsf(bf_lo(w1)));
+    m = fmaxf(m, fabsf(bf_hi(w1)));
+}
+
+// Block-wide max of a non-negative, non-NaN float; result valid in thread 0.
+__device__ __forceinline__ uint32_t block_max_bits(float m) {
+    __shared__ uint32_t warp_max[kThreads / 32];
+    uint32_t bits = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) warp_max[warp] = bits;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t v = lane < kThreads / 32 ? warp_max[lane] : 0u;
+        bits = __reduce_max_sync(0xffffffffu, v);
+    }
+    return bits;
+}
+
+template <int FMT, int MODE>
+__global__ void __launch_bounds__(kThreads)
+quantize_kernel(const uint16_t* __restrict__ x, int64_t n, uint8_t* __restrict__ out8,
+                fp8_ring* ring, uint32_t* amax_acc, float* amax_out, float* scale_out) {
+    const float fmax = fmt_max(FMT);
+    float s = 1.0f;
+    if (MODE == kDelayed) {
+        s = *reinterpret_cast<volatile float*>(&ring->scale);
+    } else if (MODE == kCurrentQuant) {
+        const float a = __uint_as_float(*reinterpret_cast<volatile uint32_t*>(amax_acc));
+        s = (a > 0.0f && isfinite(a)) ? scale_from_amax(fmax, a) : 1.0f;
+    }
+    if (MODE != kAmaxOnly && blockIdx.x == 0 && threadIdx.x == 0) *scale_out = s;
+
+    const uint4* xv = reinterpret_cast<const uint4*>(x);
+    uint2* ov = reinterpret_cast<uint2*>(out8);
+    const int64_t units = n >> 3;  // 8 elements per unit
+    const int64_t tid = int64_t(blockIdx.x) * kThreads + threadIdx.x;
+    const int64_t stride = int64_t(gridDim.x) * kThreads;
+    float m = 0.0f;
+
+    for (int64_t base = tid; base < units; base += stride * kUnroll) {
+        uint4 v[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t i = base + u * stride;
+            if (i < units) v[u] = __ldg(xv + i);
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t i = base + u * stride;
+            if (i < units) {
+                if (MODE == kAmaxOnly) {
+                    amax4(v[u].x, v[u].y, m);
+                    amax4(v[u].z, v[u].w, m);
+                } else {
+                    uint2 q;
+                    q.x = quant4<FMT>(v[u].x, v[u].y, s, m);
+                    q.y = quant4<FMT>(v[u].z, v[u].w, s, m);
+                    ov[i] = q;
+                }
+            }
+        }
+    }
+    // ragged tail (n mod 8 elements): one thread, scalar
+    if (tid == 0) {
+        for (int64_t i = units << 3; i < n; ++i) {
+            const float a = __uint_as_float(uint32_t(x[i]) << 16);
+            m = fmaxf(m, fabsf(a));
+            if (MODE != kAmaxOnly) out8[i] = uint8_t(cvt_pair<FMT>(__fmul_rn(a, s), 0.0f));
+        }
+    }
+
+    const uint32_t bits = block_max_bits(m);
+    if (threadIdx.x != 0) return;
+    uint32_t* acc = MODE == kDelayed ? &ring->amax_bits : amax_acc;
+    if (bits != 0u) atomicMax(acc, bits);
+    if (MODE != kDelayed) return;
+
+    // Last-block election: every block publishes its amax, fences, and takes a
+    // ticket; the block holding the final ticket sees every block's amax.
+    __threadfence();
+    const uint32_t ticket = atomicAdd(&ring->ticket, 1u);
+    if (ticket != gridDim.x - 1) return;
+    __threadfence();
+    const float a = __uint_as_float(atomicExch(&ring->amax_bits, 0u));
+    volatile fp8_ring* r = ring;
+    const uint32_t idx = r->idx & (FP8_RING_HISTORY - 1);
+    r->hist[idx] = a;
+    float wmax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < FP8_RING_HISTORY; ++i) wmax = fmaxf(wmax, r->hist[i]);
+    if (wmax > 0.0f && isfinite(wmax)) r->scale = scale_from_amax(fmax, wmax);
+    r->idx = (idx + 1) & (FP8_RING_HISTORY - 1);
+    if (amax_out) *amax_out = a;
+    __threadfence();
+    atomicExch(&ring->ticket, 0u);
+}
+
+__global__ void ring_write_kernel(fp8_ring* ring, fp8_ring value) {
+    const int t = threadIdx.x;
+    if (t < FP8_RING_HISTORY) ring->hist[t] = value.hist[t];
+    if (t == 0) {
+        ring->scale = value.scale;
+        ring->idx = value.idx;
+        ring->amax_bits = 0u;
+        ring->ticket = 0u;
+    }
+}
+
+int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int c = 0;
+        if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0) c = 148;
+        cached[dev] = c;
+    }
+    return cached[dev];
+}
+
+int grid_for(int64_t n) {
+    const int64_t units = n >> 3;
+    const int64_t want = (units + int64_t(kThreads) * kUnroll - 1) / (int64_t(kThreads) * kUnroll);
+    const int64_t cap = int64_t(sm_count()) * (2048 / kThreads);
+    int64_t g = want < cap ? want : cap;
+    return int(g < 1 ? 1 : g);
+}
+
+template <int FMT>
+fp8_status launch_quantize(const uint16_t* x, int64_t n, fp8_ring* ring, uint8_t* out8,
+                           float* amax_out, float* scale_out, cudaStream_t st) {
+    const int grid = grid_for(n);
+    if (ring) {
+        quantize_kernel<FMT, kDelayed><<<grid, kThreads, 0, st>>>(x, n, out8, ring, nullptr, amax_out,
+                                                                 scale_out);
+        return launch_status();
+    }
+    uint32_t* acc = reinterpret_cast<uint32_t*>(amax_out);
+    if (cudaMemsetAsync(acc, 0, sizeof(uint32_t), st) != cudaSuccess) return FP8_ERR_CUDA;
+    quantize_kernel<FMT, kAmaxOnly><<<grid, kThreads, 0, st>>>(x, n, out8, nullptr, acc, nullptr, nullptr);
+    if (launch_status() != FP8_OK) return FP8_ERR_CUDA;
+    quantize_kernel<FMT, kCurrentQuant><<<grid, kThreads, 0, st>>>(x, n, out8, nullptr, acc, nullptr,
+                                                                  scale_out);
+    return launch_status();
+}
+
+bool scale_ok(float s) { return s > 0.0f && s <= 3.402823466e38f; }
+
+}  // namespace
+}  // namespace fp8lite
+
+using namespace fp8lite;
+
+extern "C" const char* fp8_status_string(fp8_status s) {
+    switch (s) {
+        case FP8_OK: return "FP8_OK";
+        case FP8_ERR_INVALID_ARG: return "FP8_ERR_INVALID_ARG";
+        case FP8_ERR_ALIGNMENT: return "FP8_ERR_ALIGNMENT";
+        case FP8_ERR_UNSUPPORTED: return "FP8_ERR_UNSUPPORTED";
+        case FP8_ERR_CUDA: return "FP8_ERR_CUDA";
+        case FP8_ERR_DEVICE_TIMEOUT: return "FP8_ERR_DEVICE_TIMEOUT";
+    }
+    return "FP8_ERR_UNKNOWN";
+}
+
+extern "C" int fp8_abi_version(void) { return FP8LITE_ABI_VERSION; }
+
+extern "C" fp8_status fp8_ring_init(fp8_ring* ring, float init_scale, void* stream) {
+    if (!ring) return FP8_ERR_INVALID_ARG;
+    if (!aligned(ring, 4)) return FP8_ERR_ALIGNMENT;
+    if (!scale_ok(init_scale)) return FP8_ERR_INVALID_ARG;
+    fp8_ring v = {};
+    v.scale = init_scale;
+    ring_write_kernel<<<1, 32, 0, as_stream(stream)>>>(ring, v);
+    return launch_status();
+}
+
+extern "C" fp8_status fp8_ring_get(const fp8_ring* ring, fp8_ring* host, void* stream) {
+    if (!ring || !host) return FP8_ERR_INVALID_ARG;
+    if (!aligned(ring, 4)) return FP8_ERR_ALIGNMENT;
+    cudaStream_t st = as_stream(stream);
+    if (cudaMemcpyAsync(host, ring, sizeof(fp8_ring), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return FP8_ERR_CUDA;
+    return cudaStreamSynchronize(st) == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
+extern "C" fp8_status fp8_ring_set(fp8_ring* ring, const fp8_ring* host, void* stream) {
+    if (!ring || !host) return FP8_ERR_INVALID_ARG;
+    if (!aligned(ring, 4)) return FP8_ERR_ALIGNMENT;
+    if (host->idx >= FP8_RING_HISTORY || !scale_ok(host->scale)) return FP8_ERR_INVALID_ARG;
+    ring_write_kernel<<<1, 32, 0, as_stream(stream)>>>(ring, *host);
+    return launch_status();
+}
+
+extern "C" fp8_status fp8_quantize(const void* x, int64_t n, fp8_fmt fmt, fp8_ring* ring, uint8_t* out8,
+                                   float* amax_out, float* scale_out, void* stream) {
+    if (!valid_fmt(fmt)) return FP8_ERR_INVALID_ARG;
+    if (n < 0 || n >= (int64_t(1) << 40)) return FP8_ERR_INVALID_ARG;
+    if (!scale_out) return FP8_ERR_INVALID_ARG;
+    if (n > 0 && (!x || !out8)) return FP8_ERR_INVALID_ARG;
+    if (!ring && !amax_out) return FP8_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(out8, 16)) return FP8_ERR_ALIGNMENT;
+    if (ring && !aligned(ring, 4)) return FP8_ERR_ALIGNMENT;
+    if (!aligned(scale_out, 4) || !aligned(amax_out, 4)) return FP8_ERR_ALIGNMENT;
+    const uint16_t* xb = static_cast<const uint16_t*>(x);
+    cudaStream_t st = as_stream(stream);
+    return fmt == FP8_E4M3 ? launch_quantize<FP8_E4M3>(xb, n, ring, out8, amax_out, scale_out, st)
+                           : launch_quantize<FP8_E5M2>(xb, n, ring, out8, amax_out, scale_out, st);
+}

@@ -1,0 +1,182 @@
+/*
+ * fp8lite -- per-tensor FP8 quantization with delayed scaling, and the
+ * per-tensor-scaled FP8 GEMM of a linear layer, for NVIDIA B200 (sm_100a).
+ *
+ * The C ABI of the library. Plain pointers and sizes only; the caller owns
+ * every buffer (device memory unless stated) and the library allocates
+ * nothing per call. All compute calls are asynchronous and stream-ordered on
+ * `stream` (a cudaStream_t passed as void*; NULL is the legacy default
+ * stream) and do no host synchronisation, so a sequence of them can be
+ * captured into a CUDA graph. Arguments are validated on the host BEFORE any
+ * launch; a rejected call launches nothing and returns a non-OK status.
+ *
+ * Method sources (AstrAI FP8 commit logs):
+ *  [fp8.py@4dc5e923]  astrai/extension/fp8.py, commit 4dc5e923
+ *  [fp8.py@f4c44ebf]  astrai/extension/fp8.py, commit f4c44ebf
+ *  [mma@cebdd45d]     tests/extension/test_fp8_mma.py, commit cebdd45d
+ *  [gemm@5e76fbd1]    csrc/kernels/fp8/gemm.cuh, commit 5e76fbd1
+ * FP8 formats: OCP 8-bit floating point specification (OFP8) rev. 1.0.
+ */
+#ifndef FP8LITE_H
+#define FP8LITE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FP8LITE_ABI_VERSION 1
+
+/* Exported entry points (the library is built with hidden visibility). */
+#if defined(__GNUC__)
+#define FP8LITE_API __attribute__((visibility("default")))
+#else
+#define FP8LITE_API
+#endif
+
+/* FP8 encodings (OFP8): E4M3 = the "FN" variant, max 448, no Inf;
+ * E5M2 = IEEE-like, max 57344. The pages use E4M3 for activations and
+ * weights and E5M2 for gradients [fp8.py@4dc5e923, bullet on the fp8
+ * backward regression test]. */
+typedef enum fp8_fmt { FP8_E4M3 = 0, FP8_E5M2 = 1 } fp8_fmt;
+
+/* GEMM layouts, BLAS-style op tags on row-major storage
+ * [gemm@5e76fbd1, bullet on RowMajor/ColMajor operand tags]:
+ *   FP8_NT: A [M,K], B [N,K]  C = A * B^T   (forward  y  = x W^T)
+ *   FP8_NN: A [M,K], B [K,N]  C = A * B     (backward dX = g W)
+ *   FP8_TN: A [K,M], B [K,N]  C = A^T * B   (backward dW = g^T x) */
+typedef enum fp8_layout { FP8_NT = 0, FP8_NN = 1, FP8_TN = 2 } fp8_layout;
+
+typedef enum fp8_status {
+    FP8_OK = 0,
+    FP8_ERR_INVALID_ARG = 1,    /* bad enum, null required pointer, bad size */
+    FP8_ERR_ALIGNMENT = 2,      /* base or stride not aligned as documented */
+    FP8_ERR_UNSUPPORTED = 3,    /* shape or option this build cannot run */
+    FP8_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed */
+    FP8_ERR_DEVICE_TIMEOUT = 5  /* a bounded device wait gave up (GEMM) */
+} fp8_status;
+
+/* Delayed-scaling amax history of ONE tensor role (x, W or g of one linear)
+ * [fp8.py@4dc5e923, bullets on _ScaleRing and the three rings per linear].
+ * Device-resident, caller-allocated (FP8_RING_BYTES, 4-byte aligned).
+ *   hist[16]   amax of the last 16 calls (fp32), written at hist[idx]
+ *   scale      the scale the NEXT call quantizes with (multiplier into FP8)
+ *   idx        next slot of hist, 0..15
+ *   amax_bits  in-flight amax accumulator; 0 between calls
+ *   ticket     last-block election counter; 0 between calls
+ * One ring must not be used by two calls that overlap on the GPU. */
+#define FP8_RING_HISTORY 16
+typedef struct fp8_ring {
+    float hist[FP8_RING_HISTORY];
+    float scale;
+    uint32_t idx;
+    uint32_t amax_bits;
+    uint32_t ticket;
+} fp8_ring;
+#define FP8_RING_BYTES 80
+
+/* Human-readable name of a status (static string). */
+FP8LITE_API const char* fp8_status_string(fp8_status s);
+
+/* FP8LITE_ABI_VERSION of the built library. */
+FP8LITE_API int fp8_abi_version(void);
+
+/* Reset a ring: hist = 0, idx = 0, scale = init_scale, accumulators 0.
+ * init_scale must be finite and > 0 (the plain reading starts at 1.0).
+ * Asynchronous on `stream` (one tiny kernel, graph-capturable). */
+FP8LITE_API fp8_status fp8_ring_init(fp8_ring* ring, float init_scale, void* stream);
+
+/* Checkpoint: copy the ring to host memory `host` (FP8_RING_BYTES).
+ * Synchronises `stream` before returning. */
+FP8LITE_API fp8_status fp8_ring_get(const fp8_ring* ring, fp8_ring* host, void* stream);
+
+/* Restore: write the host copy `host` into the device ring (asynchronous,
+ * by value, no host sync). idx must be < 16 and scale finite and > 0; the
+ * accumulators are reset to 0 whatever `host` holds. */
+FP8LITE_API fp8_status fp8_ring_set(fp8_ring* ring, const fp8_ring* host, void* stream);
+
+/* Per-tensor quantization of n bf16 values x -> n FP8 codes out8, with the
+ * amax measured on the UNQUANTIZED input [fp8.py@4dc5e923, bullets on the
+ * amax bug].
+ *
+ *   q_i = sat_rne_fmt( fp32(x_i * s) )   (fp32 product, then one FP8
+ *   rounding to nearest-even; magnitudes above the format's max saturate)
+ *
+ * ring != NULL -- delayed scaling, ONE kernel launch: s = ring->scale as it
+ *   stood before the call; the last thread block to finish (threadfence +
+ *   ticket election) writes amax into hist[idx], advances idx, takes the max
+ *   of the window and publishes ring->scale = fmt_max / max when that max is
+ *   finite and > 0 (otherwise the scale is kept), then resets the ring's
+ *   accumulators [fp8.py@4dc5e923, bullet on the last-block epilogue].
+ * ring == NULL -- current ("dynamic") scaling [fp8.py@4dc5e923, bullet on
+ *   the dynamic path]: s = fmt_max / amax(x) (1 if amax is 0 or not finite);
+ *   a memset and two launches (amax pass, quantize pass).
+ * fmt_max / m is an IEEE fp32 division; an overflow is clamped to FLT_MAX.
+ *
+ * x          device, bf16[n], 16-byte aligned
+ * n          element count, 0 <= n < 2^40 (n = 0 folds amax 0)
+ * out8       device, uint8[n], 16-byte aligned, FP8 codes of `fmt`
+ * amax_out   device float: amax(x). Optional (NULL) with a ring; REQUIRED
+ *            without one (it is the accumulator of the amax pass)
+ * scale_out  device float, REQUIRED: the scale s this call used. A GEMM on
+ *            out8 must dequantize with THIS value, not with ring->scale,
+ *            which the call has already replaced [fp8.py@f4c44ebf, bullet on
+ *            snapshotting sx/sw/sg before the finalize].
+ * Errors: FP8_ERR_INVALID_ARG (bad fmt, NULL x/out8/scale_out with n > 0,
+ *         NULL amax_out without a ring, n out of range),
+ *         FP8_ERR_ALIGNMENT (x or out8 not 16-byte aligned, ring not 4-byte
+ *         aligned), FP8_ERR_CUDA (launch failure). */
+FP8LITE_API fp8_status fp8_quantize(const void* x, int64_t n, fp8_fmt fmt, fp8_ring* ring,
+                        uint8_t* out8, float* amax_out, float* scale_out,
+                        void* stream);
+
+/* Per-tensor-scaled FP8 GEMM with fused bias and bf16 output
+ * [fp8.py@f4c44ebf, bullets on the fused bias and 3-D operands;
+ *  mma@cebdd45d, bullet on the bias_scale slot].
+ *
+ *   out[b,i,j] = bf16_rne( (sum_k op(A_b)[i,k] op(B_b)[k,j]) / (sa*sb) + bias_j )
+ *
+ * accumulated in fp32 on the tensor cores, the scale and the bias applied in
+ * fp32, then ONE rounding to bf16. bias_j is bias[j] (bf16) when bias_scale
+ * is NULL, dec(bias[j]) / *bias_scale (fp8 codes of bias_fmt) when it is not,
+ * 0 when bias is NULL; the bias is broadcast over rows and batches.
+ *
+ * a8, b8     device FP8 codes of formats fa, fb in `layout` (see fp8_layout),
+ *            each 16-byte aligned
+ * sa, sb     device floats: the scales the operands were quantized with
+ *            (the scale_out of fp8_quantize)
+ * M, N, K    >= 1 each. The contiguous dimension of every operand must be a
+ *            multiple of 16 elements (TMA row pitch): K for A in NT/NN and
+ *            B in NT; N for B in NN/TN; M for A in TN. M and N are otherwise
+ *            free (M = 1 and N = 7 are valid).
+ * batch      >= 1; stride_a / stride_b / stride_c in ELEMENTS between
+ *            consecutive batches; stride_a or stride_b = 0 broadcasts one
+ *            matrix to every batch; nonzero operand strides must be multiples
+ *            of 16; stride_c >= M*N when batch > 1.
+ * bias       NULL, device bf16[N], or device FP8 codes[N] of bias_fmt
+ * bias_scale NULL (bf16 bias) or device float (FP8 bias)
+ * out        device bf16[batch*stride_c], row-major [M,N] per batch,
+ *            4-byte aligned
+ * Errors: FP8_ERR_INVALID_ARG, FP8_ERR_ALIGNMENT as listed above,
+ *         FP8_ERR_UNSUPPORTED (a size >= 2^31 per matrix dimension),
+ *         FP8_ERR_CUDA. A bounded device wait that gives up does not fail
+ *         the call; it is reported by fp8_last_device_error. */
+FP8LITE_API fp8_status fp8_mm(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8, fp8_fmt fb,
+                  const float* sa, const float* sb, fp8_layout layout,
+                  int64_t M, int64_t N, int64_t K, int64_t batch,
+                  int64_t stride_a, int64_t stride_b, int64_t stride_c,
+                  const void* bias, const float* bias_scale, fp8_fmt bias_fmt,
+                  void* out, void* stream);
+
+/* Synchronises the current device, then reads and clears the library's
+ * device error word: FP8_ERR_DEVICE_TIMEOUT if a GEMM thread block gave up a
+ * bounded wait since the last call (its output tile is then undefined),
+ * FP8_OK otherwise, FP8_ERR_CUDA if the synchronisation failed. */
+FP8LITE_API fp8_status fp8_last_device_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8LITE_H */

@@ -1,0 +1,106 @@
+"""The C-ABI library loads, exports every declared entry point, and rejects
+bad arguments on the host before any launch (CPU only: no compute call)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def fp8():
+    from fp8_delayed_scaling_quantize_b200 import build
+    build.build()
+    import fp8_delayed_scaling_quantize_b200 as m
+    return m
+
+
+def _declared():
+    with open(os.path.join(ROOT, "include", "fp8lite.h")) as f:
+        text = f.read()
+    return re.findall(r"FP8LITE_API\s+[\w\s\*]+?\b(fp8_\w+)\s*\(", text)
+
+
+def test_every_declared_symbol_is_exported(fp8):
+    names = _declared()
+    assert len(names) >= 8
+    lib = ctypes.CDLL(fp8.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_abi_version_and_status_strings(fp8):
+    assert fp8.fp8_abi_version() == 1
+    for code, name in [(0, "FP8_OK"), (1, "FP8_ERR_INVALID_ARG"), (2, "FP8_ERR_ALIGNMENT"),
+                       (3, "FP8_ERR_UNSUPPORTED"), (4, "FP8_ERR_CUDA"), (5, "FP8_ERR_DEVICE_TIMEOUT")]:
+        assert fp8.status_string(code) == name
+
+
+# Fake device addresses: the host validation must reject before touching them.
+A = 0x7F0000000000
+S = 0x7F0000100000
+
+
+def q(fp8, x=A, n=64, fmt=0, ring=None, out=A + 4096, amax=S, scale=S + 4):
+    return fp8.raw_status("fp8_quantize", x, n, fmt, ring, out, amax, scale, None)
+
+
+def test_quantize_validation(fp8):
+    assert q(fp8, fmt=2) == fp8.FP8_ERR_INVALID_ARG
+    assert q(fp8, fmt=-1) == fp8.FP8_ERR_INVALID_ARG
+    assert q(fp8, n=-1) == fp8.FP8_ERR_INVALID_ARG
+    assert q(fp8, n=1 << 40) == fp8.FP8_ERR_INVALID_ARG
+    assert q(fp8, scale=None) == fp8.FP8_ERR_INVALID_ARG
+    assert q(fp8, x=None) == fp8.FP8_ERR_INVALID_ARG
+    assert q(fp8, out=None) == fp8.FP8_ERR_INVALID_ARG
+    assert q(fp8, amax=None) == fp8.FP8_ERR_INVALID_ARG  # current scaling needs it
+    assert q(fp8, x=A + 2) == fp8.FP8_ERR_ALIGNMENT
+    assert q(fp8, out=A + 4096 + 8) == fp8.FP8_ERR_ALIGNMENT
+    assert q(fp8, ring=S + 2) == fp8.FP8_ERR_ALIGNMENT
+    assert q(fp8, scale=S + 1) == fp8.FP8_ERR_ALIGNMENT
+
+
+def mm(fp8, a8=A, fa=0, b8=A + 65536, fb=0, sa=S, sb=S + 4, layout=0, M=128, N=128, K=128,
+       batch=1, stride_a=0, stride_b=0, stride_c=0, bias=None, bias_scale=None, bias_fmt=0,
+       out=A + 262144):
+    return fp8.raw_status("fp8_mm", a8, fa, b8, fb, sa, sb, layout, M, N, K, batch, stride_a,
+                          stride_b, stride_c, bias, bias_scale, bias_fmt, out, None)
+
+
+def test_mm_validation(fp8):
+    E, AL, U = fp8.FP8_ERR_INVALID_ARG, fp8.FP8_ERR_ALIGNMENT, fp8.FP8_ERR_UNSUPPORTED
+    assert mm(fp8, fa=3) == E
+    assert mm(fp8, layout=3) == E
+    assert mm(fp8, a8=None) == E
+    assert mm(fp8, sa=None) == E
+    assert mm(fp8, out=None) == E
+    assert mm(fp8, M=0) == E and mm(fp8, N=0) == E and mm(fp8, K=0) == E
+    assert mm(fp8, batch=0) == E
+    assert mm(fp8, stride_a=-16, batch=2, stride_c=128 * 128) == E
+    assert mm(fp8, bias_scale=S + 8) == E            # a scale without a bias
+    assert mm(fp8, batch=2, stride_c=100) == E       # overlapping outputs
+    assert mm(fp8, M=1 << 31) == U
+    # TMA row pitch: K (NT), N for B (NN/TN), M for A (TN) multiples of 16
+    assert mm(fp8, K=100) == AL
+    assert mm(fp8, layout=1, N=100) == AL
+    assert mm(fp8, layout=2, M=100) == AL
+    assert mm(fp8, a8=A + 8) == AL
+    assert mm(fp8, batch=2, stride_a=8, stride_c=1 << 20) == AL
+    assert mm(fp8, out=A + 262144 + 2) == AL
+    # free dimensions: M and N in NT need no alignment (checked up to launch:
+    # every check above must fail before any CUDA call on this CPU-only host)
+
+
+def test_ring_validation(fp8):
+    assert fp8.raw_status("fp8_ring_init", None, ctypes.c_float(1.0), None) == fp8.FP8_ERR_INVALID_ARG
+    assert fp8.raw_status("fp8_ring_init", S, ctypes.c_float(0.0), None) == fp8.FP8_ERR_INVALID_ARG
+    assert fp8.raw_status("fp8_ring_init", S, ctypes.c_float(float("inf")), None) == fp8.FP8_ERR_INVALID_ARG
+    assert fp8.raw_status("fp8_ring_init", S + 2, ctypes.c_float(1.0), None) == fp8.FP8_ERR_ALIGNMENT
+    host = fp8.fp8_ring()
+    host.idx = 16
+    host.scale = 1.0
+    assert fp8.raw_status("fp8_ring_set", S, ctypes.byref(host), None) == fp8.FP8_ERR_INVALID_ARG
+    assert fp8.raw_status("fp8_ring_get", None, ctypes.byref(host), None) == fp8.FP8_ERR_INVALID_ARG

@@ -1,0 +1,191 @@
+"""GPU parity of fp8_quantize (through the C ABI) against the CPU oracle.
+
+Bar: bit-exact codes, amax, scale used and full ring state. NaN inputs are
+excluded from the code comparison (the NaN reading is unpinned) but must map
+to a NaN code.
+"""
+
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import E4M3, E5M2
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+@pytest.fixture(scope="module")
+def g():
+    import gpu_util
+    return gpu_util
+
+
+def _nan_code(c, fmt):
+    return (c & 0x7F) == 0x7F if fmt == E4M3 else (c & 0x7F) > 0x7C
+
+
+@pytest.mark.parametrize("fmt", [E4M3, E5M2])
+def test_every_bf16_pattern_under_many_scales(g, fmt):
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    xs = W.bf16_bit_patterns()
+    xf = xs.float().numpy()
+    finite = np.isfinite(xf)
+    xd = xs.cuda()
+    scales = [1.0, float(np.float32(448.0) / np.float32(3.0)), 2.0 ** -20, 1e-3, 3.0e38, 7.5,
+              2.0 ** 40, float(np.nextafter(np.float32(1.0), np.float32(0.0)))]
+    for s in scales:
+        s32 = np.float32(s)
+        ring = g.new_ring()
+        host = fp8.fp8_ring()
+        host.scale = float(s32)
+        fp8.fp8_ring_set(ring, host)
+        q, amax, scale = g.quantize(xd, fmt, ring)
+        got = g.codes(q)
+        want = oracle.quantize_with_scale(xf, s32, fmt)
+        nan = np.isnan(xf)
+        assert np.array_equal(got[~nan], want[~nan]), f"scale {s}"
+        assert all(_nan_code(int(c), fmt) for c in got[nan])
+        assert g.f32(scale)[0] == s32
+        assert g.f32(amax)[0] == oracle.amax(xf)          # inf: the patterns hold +-inf
+        hist, rs, idx, acc, ticket = g.ring_state(ring)
+        assert hist[0] == np.inf and idx == 1 and acc == 0 and ticket == 0
+        assert rs == s32                                   # non-finite window max keeps it
+    # finite patterns only: the ring publishes fmt_max / amax
+    ring = g.new_ring()
+    xfin = xs[torch.from_numpy(finite)].contiguous()
+    q, amax, scale = g.quantize(xfin.cuda(), fmt, ring)
+    ref = oracle.DelayedRing()
+    want, a, s = ref.step(xfin.float().numpy(), fmt)
+    assert np.array_equal(g.codes(q), want)
+    hist, rs, idx, _, _ = g.ring_state(ring)
+    assert np.array_equal(hist, ref.hist) and rs == ref.scale and idx == ref.idx
+
+
+@pytest.mark.parametrize("fmt", [E4M3, E5M2])
+@pytest.mark.parametrize("n", [0, 1, 7, 8, 15, 16, 17, 1000, 4096 * 37 + 5, (1 << 20) + 3])
+def test_current_scaling_ragged_sizes(g, fmt, n):
+    x = W.bf16_normal((n,), 0.7, 9000 + n)
+    q, amax, scale = g.quantize(x.cuda(), fmt, None)
+    want, a, s = oracle.quantize_current(x.float().numpy(), fmt)
+    assert np.array_equal(g.codes(q), want)
+    assert g.f32(amax)[0] == a
+    assert g.f32(scale)[0] == s
+
+
+def test_current_scaling_degenerate(g):
+    z = torch.zeros(1000, dtype=torch.bfloat16)
+    q, amax, scale = g.quantize(z.cuda(), E4M3, None)
+    assert g.f32(amax)[0] == 0.0 and g.f32(scale)[0] == 1.0 and not g.codes(q).any()
+    # smallest bf16 subnormal: 448 / 2^-133 overflows -> FLT_MAX
+    t = torch.tensor([2.0 ** -133, 0.0], dtype=torch.bfloat16)
+    q, amax, scale = g.quantize(t.cuda(), E4M3, None)
+    want, a, s = oracle.quantize_current(t.float().numpy(), E4M3)
+    assert g.f32(scale)[0] == s == np.finfo(np.float32).max
+    assert np.array_equal(g.codes(q), want)
+
+
+def test_ring_hand_table_on_gpu(g):
+    with open(os.path.join(GOLDEN, "ring_sequence.json")) as f:
+        gold = json.load(f)
+    ring = g.new_ring()
+    for a, used, published, why in gold["steps"]:
+        x = torch.tensor([a, -a / 2, a / 4, 0.0] * 1000, dtype=torch.bfloat16).cuda()
+        _, amax, scale = g.quantize(x, gold["fmt"], ring)
+        assert g.f32(amax)[0] == a, why
+        assert g.f32(scale)[0] == np.float32(used), why
+        assert g.ring_state(ring)[1] == np.float32(published), why
+    assert g.ring_state(ring)[2] == gold["final_idx"]
+
+
+def test_linear_stack_delayed_eight_steps(g):
+    """Every x, W, g of the dim-1024 linear stack at 2048 tokens, 8 delayed
+    steps with the per-step magnitude walk: codes, amax, scales and rings."""
+    walk = W.stack_walk()
+    rings = [[g.new_ring() for _ in range(3)] for _ in W.LINEARS]
+    refs = [[oracle.DelayedRing() for _ in range(3)] for _ in W.LINEARS]
+    rng = np.random.default_rng(1)
+    for step in range(W.STACK_STEPS):
+        tensors = W.stack_tensors(step, walk)
+        for li, t in enumerate(tensors):
+            for ri, (role, fmt) in enumerate((("x", E4M3), ("w", E4M3), ("g", E5M2))):
+                xc = t[role].reshape(-1)
+                q, amax, scale = g.quantize(xc.cuda(), fmt, rings[li][ri])
+                xf = xc.float().numpy()
+                s_used = np.float32(refs[li][ri].scale)
+                a = oracle.amax(xf)
+                refs[li][ri].fold(a, fmt)
+                got = g.codes(q)
+                if step == 0:
+                    idx = slice(None)
+                else:
+                    idx = rng.integers(0, xf.size, 200_000)
+                assert np.array_equal(got[idx], oracle.quantize_with_scale(xf[idx], s_used, fmt)), (step, li, role)
+                assert g.f32(amax)[0] == a and g.f32(scale)[0] == s_used
+                hist, rs, ridx, acc, ticket = g.ring_state(rings[li][ri])
+                assert np.array_equal(hist, refs[li][ri].hist) and rs == refs[li][ri].scale
+                assert ridx == refs[li][ri].idx and acc == 0 and ticket == 0
+
+
+def test_graph_replay_and_checkpoint(g):
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    n = 3 * (1 << 18) + 11
+    base = W.bf16_normal((n,), 1.0, 77).cuda()
+    x = base.clone()
+    ring = g.new_ring()
+    out = torch.empty(n, dtype=torch.uint8, device="cuda")
+    amax = torch.empty(1, device="cuda")
+    scale = torch.empty(1, device="cuda")
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            fp8.fp8_quantize(x, n, E4M3, ring, out, amax, scale, stream=stream)
+    torch.cuda.synchronize()
+    fp8.fp8_ring_init(ring, 1.0)
+    ref = oracle.DelayedRing()
+    factors = W.uniform(0.5, 2.0, 78, 20)
+    saved = None
+    for i in range(20):
+        x.copy_((base.float() * float(factors[i]) * (i + 1)).to(torch.bfloat16))
+        torch.cuda.synchronize()
+        graph.replay()
+        torch.cuda.synchronize()
+        want, a, s = ref.step(x.float().cpu().numpy(), E4M3)
+        assert np.array_equal(g.codes(out), want), i
+        assert g.f32(scale)[0] == s and g.f32(amax)[0] == a
+        if i == 9:
+            saved = fp8.fp8_ring_get(ring)
+            saved_ref = ref.copy()
+    # restore the step-9 checkpoint into a fresh ring and continue: identical
+    ring2 = g.new_ring()
+    fp8.fp8_ring_set(ring2, saved)
+    x.copy_((base.float() * 3.0).to(torch.bfloat16))
+    q2, _, s2 = g.quantize(x, E4M3, ring2)
+    want, _, s = saved_ref.step(x.float().cpu().numpy(), E4M3)
+    assert g.f32(s2)[0] == s and np.array_equal(g.codes(q2), want)
+    del graph
+
+
+def test_empty_input_folds_zero(g):
+    ring = g.new_ring(2.5)
+    q, amax, scale = g.quantize(torch.empty(0, dtype=torch.bfloat16, device="cuda"), E4M3, ring)
+    hist, rs, idx, _, _ = g.ring_state(ring)
+    assert g.f32(amax)[0] == 0.0 and g.f32(scale)[0] == np.float32(2.5)
+    assert idx == 1 and rs == np.float32(2.5) and not hist.any()
+
+
+def test_misaligned_input_is_rejected(g):
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    x = torch.zeros(64, dtype=torch.bfloat16, device="cuda")
+    out = torch.empty(64, dtype=torch.uint8, device="cuda")
+    amax = torch.empty(1, device="cuda")
+    st = fp8.raw_status("fp8_quantize", x.data_ptr() + 2, 32, 0, None, out.data_ptr(),
+                        amax.data_ptr(), amax.data_ptr(), None)
+    assert st == fp8.FP8_ERR_ALIGNMENT
