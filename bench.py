@@ -1,0 +1,583 @@
+"""Benchmark of the FP8 linear-layer hot path on B200.
+
+One step = one pass of the whole path over the dim-1024 transformer linear
+stack at 2048 tokens (B4 x T512): for each of the 4 linears (QKV 1024->3072,
+out 1024->1024, MLP 1024->4096, 4096->1024) delayed-scaling quantize of x
+and W to E4M3 and of the gradient g to E5M2 (ring finalized in-kernel),
+then the forward NT GEMM y = x W^T, the dX NN GEMM g W and the dW TN GEMM
+g^T x -- 12 quantize launches and 12 GEMM launches, all through the C ABI.
+
+value  = GEMM FLOPs of the step (154.6 GFLOP) / device step time, TFLOP/s,
+         the step replayed as one CUDA graph (24 kernel nodes), inputs
+         resident in HBM, rotating through 3 input sets (276 MB > 126 MB L2).
+e2e    = the same metric through the public API with HOST buffers: pinned
+         host -> device copies of x, W, g and device -> host copies of y,
+         dX, dW inside the timed region, eager calls.
+roofline / roofline_quantize = the GEMM kernel and the quantize kernel,
+         each timed per launch with CUDA events on the launching stream.
+cpu_baseline = the CPU oracle (numpy, fp64 GEMM) on one full step.
+
+--impl reference times the oracle on the host cores instead (a bounded
+sample of the same step per bench step).
+"""
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "FP8 GEMM TFLOP/s & quantize GB/s on 1 B200, % of roofline"
+WORKLOAD = "linear stack dim1024 tokens2048 (B4xT512): QKV/out/MLP-up/MLP-down, fwd NT + dX NN + dW TN, delayed rings H=16"
+N_SETS = 3
+E4M3, E5M2 = 0, 1
+NT, NN, TN = 0, 1, 2
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------ distributed ---
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------- clocks ---
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    NAMES = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+             0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+             0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index, period=0.01):
+        self.period = period
+        self.samples = []
+        self.reasons = 0
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.ok:
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"], "samples": 0}
+        names = [n for bit, n in self.NAMES.items() if self.reasons & bit]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------- the stack ---
+
+class Stack:
+    """Device buffers and the 24 C-ABI calls of one step of the linear stack."""
+
+    def __init__(self, fp8, n_sets=N_SETS, dev="cuda"):
+        self.fp8 = fp8
+        self.dev = dev
+        self.sets = []
+        for s in range(n_sets):
+            ts = W.stack_tensors(s)
+            self.sets.append([{k: v.to(dev) for k, v in t.items()} for t in ts])
+        T = W.TOKENS
+        self.lin = []
+        for li, (name, d_in, d_out) in enumerate(W.LINEARS):
+            L = {"name": name, "d_in": d_in, "d_out": d_out}
+            L["q"] = {r: torch.empty(n, dtype=torch.uint8, device=dev)
+                      for r, n in (("x", T * d_in), ("w", d_out * d_in), ("g", T * d_out))}
+            L["ring"] = {r: torch.empty(20, dtype=torch.int32, device=dev) for r in ("x", "w", "g")}
+            for r in L["ring"].values():
+                fp8.fp8_ring_init(r, 1.0)
+            L["scale"] = {r: torch.empty(1, device=dev) for r in ("x", "w", "g")}
+            L["amax"] = {r: torch.empty(1, device=dev) for r in ("x", "w", "g")}
+            L["y"] = torch.empty(T * d_out, dtype=torch.bfloat16, device=dev)
+            L["dx"] = torch.empty(T * d_in, dtype=torch.bfloat16, device=dev)
+            L["dw"] = torch.empty(d_out * d_in, dtype=torch.bfloat16, device=dev)
+            self.lin.append(L)
+        self.flops = W.stack_flops()
+        self.q_elems = W.stack_quant_elems()
+
+    def quant_calls(self, s, li):
+        L, t = self.lin[li], self.sets[s][li]
+        return [(t[r], t[r].numel(), fmt, L["ring"][r], L["q"][r], L["amax"][r], L["scale"][r])
+                for r, fmt in (("x", E4M3), ("w", E4M3), ("g", E5M2))]
+
+    def gemm_calls(self, li):
+        L = self.lin[li]
+        T, di, do = W.TOKENS, L["d_in"], L["d_out"]
+        q, sc = L["q"], L["scale"]
+        return [
+            # forward y = x W^T: NT, M=T, N=d_out, K=d_in
+            (q["x"], E4M3, q["w"], E4M3, sc["x"], sc["w"], NT, T, do, di, 1, 0, 0, 0, None, None, 0, L["y"]),
+            # dX = g W: NN, M=T, N=d_in, K=d_out
+            (q["g"], E5M2, q["w"], E4M3, sc["g"], sc["w"], NN, T, di, do, 1, 0, 0, 0, None, None, 0, L["dx"]),
+            # dW = g^T x: TN, M=d_out, N=d_in, K=T
+            (q["g"], E5M2, q["x"], E4M3, sc["g"], sc["x"], TN, do, di, T, 1, 0, 0, 0, None, None, 0, L["dw"]),
+        ]
+
+    def gemm_flops(self, li):
+        L = self.lin[li]
+        return 2 * W.TOKENS * L["d_in"] * L["d_out"]
+
+    def step(self, s, stream, events=None):
+        """Issue one step on input set s. With `events`, record a CUDA event
+        pair around every launch: events[kind] += [(start, end, units)]."""
+        fp8 = self.fp8
+        for li in range(len(self.lin)):
+            for args in self.quant_calls(s, li):
+                if events is not None:
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                fp8.fp8_quantize(*args, stream=stream)
+                if events is not None:
+                    e1.record(stream)
+                    events["quantize"].append((e0, e1, args[1]))
+            for args in self.gemm_calls(li):
+                if events is not None:
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                fp8.fp8_mm(*args, stream=stream)
+                if events is not None:
+                    e1.record(stream)
+                    events["gemm"].append((e0, e1, self.gemm_flops(li), args[6], args[7:10]))
+
+
+def hold_stream(stream, us=2000):
+    """Park the stream in a device-side sleep while the host enqueues the
+    next launches, so that event pairs around each launch time the kernel,
+    not the host's submission gaps."""
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(int(us * 1965))
+
+
+def gemm_algorithmic_bytes(layout, M, N, K):
+    """Compulsory HBM bytes of one GEMM launch: operands once, bf16 out once."""
+    return M * K + N * K + 2 * M * N
+
+
+# ------------------------------------------------------------ our arm -------
+
+def run_ours(args, world, rank, local):
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    hbm, bf16_burst, bf16_sust, peak_src = _peaks()
+    fp8_burst = 2.0 * bf16_burst      # dense FP8 = 2x dense bf16 (nominal 4.5 / 2.25 PF/s)
+    stream = torch.cuda.Stream()
+    stack = Stack(fp8)
+    torch.cuda.synchronize()
+
+    # warm-up (eager) also sets kernel attributes before any capture
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):
+            stack.step(i % N_SETS, stream)
+    torch.cuda.synchronize()
+
+    graphs = []
+    if not args.no_graph:
+        for s in range(N_SETS):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                stack.step(s, stream)
+            graphs.append(g)
+        torch.cuda.synchronize()
+        for i in range(max(args.warmup, 3)):
+            with torch.cuda.stream(stream):
+                graphs[i % N_SETS].replay()
+        torch.cuda.synchronize()
+
+    # ---- timed region -------------------------------------------------
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for i in range(args.steps):
+                if graphs:
+                    graphs[i % N_SETS].replay()
+                else:
+                    stack.step(i % N_SETS, stream)
+            e1.record(stream)
+        e1.synchronize()
+    torch.cuda.synchronize()
+    barrier(world)
+    t_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    ms_step = t_ms / args.steps
+    value = stack.flops * args.steps * world / (t_ms * 1e-3) / 1e12
+
+    # ---- per-kernel breakdown -----------------------------------------
+    # Each of the step's 24 launches is repeated back to back between one
+    # event pair (the stream held while the host enqueues), so the average is
+    # the kernel's steady-state cost on the stream, as inside the graph.
+    q_ms = g_ms = 0.0
+    q_elems = g_flops = g_bytes = 0
+    n_g = n_q = 0
+    per_shape = {}
+    reps = args.breakdown_reps
+    for li in range(len(stack.lin)):
+        calls = [("quantize", c) for c in stack.quant_calls(0, li)] + [("gemm", c) for c in stack.gemm_calls(li)]
+        for kind, c in calls:
+            fn = fp8.fp8_quantize if kind == "quantize" else fp8.fp8_mm
+            hold_stream(stream)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                fn(*c, stream=stream)
+            e1.record(stream)
+            e1.synchronize()
+            ms = e0.elapsed_time(e1) / reps
+            if kind == "quantize":
+                q_ms += ms
+                q_elems += c[1]
+                n_q += 1
+            else:
+                M, N, K = c[7:10]
+                g_ms += ms
+                g_flops += 2 * M * N * K
+                g_bytes += gemm_algorithmic_bytes(c[6], M, N, K)
+                n_g += 1
+                per_shape[f"{'NT NN TN'.split()[c[6]]} {M}x{N}x{K}"] = (ms, 2 * M * N * K)
+    gemm_tf = g_flops / (g_ms * 1e-3) / 1e12
+    quant_gbs = 3.0 * q_elems / (q_ms * 1e-3) / 1e9
+    gemm_detail = {k: {"us": round(1e3 * ms, 2), "tflops": round(f / (ms * 1e-3) / 1e12, 1)}
+                   for k, (ms, f) in per_shape.items()}
+
+    # ---- e2e: host buffers through the public API ------------------------
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(fp8, stack, stream, args.e2e_steps, world)
+        e2e["value"] = round(e2e["value"], 3)
+
+    gpu_launches = 24 * args.steps
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8 e4m3/e5m2 operands, fp32 accumulate, bf16 out",
+        "data": "synthetic (seeded bf16 normals of the workload's shapes)",
+        "config": {"workload": WORKLOAD, "tokens": W.TOKENS, "linears": [list(l[1:]) for l in W.LINEARS],
+                   "gemm_gflop_per_step": round(stack.flops / 1e9, 2),
+                   "quant_elems_per_step": stack.q_elems,
+                   "l2": f"{N_SETS} rotating input sets ({N_SETS * 2 * stack.q_elems / 1e6:.0f} MB bf16) > 126 MB L2",
+                   "launch": "CUDA graph per step" if graphs else "eager",
+                   "parallelism": f"replicas x{world}"},
+        "quantize_gbs": round(quant_gbs, 1),
+        "roofline": {"bound": "tensor", "achieved": round(gemm_tf, 1), "peak": round(fp8_burst, 1),
+                     "unit": "TFLOP/s", "frac": round(gemm_tf / fp8_burst, 4),
+                     "traffic": None,
+                     "kernel": "fp8_gemm_kernel (all 12 GEMM launches of a step, FLOP-weighted)",
+                     "peak_source": f"{peak_src}: 2 x bf16 burst {bf16_burst} TF/s (nominal fp8:bf16 = 2)",
+                     "algorithmic_bytes_per_launch": round(g_bytes / n_g),
+                     "flops_per_launch": round(g_flops / n_g),
+                     "avg_launch_us": round(1e3 * g_ms / n_g, 2)},
+        "roofline_quantize": {"bound": "hbm", "achieved": round(quant_gbs, 1), "peak": hbm, "unit": "GB/s",
+                              "frac": round(quant_gbs / hbm, 4), "traffic": None,
+                              "kernel": "quantize_kernel (delayed, 12 launches per step)",
+                              "peak_source": f"{peak_src} hbm copy",
+                              "algorithmic_bytes_per_launch": round(3 * q_elems / n_q),
+                              "avg_launch_us": round(1e3 * q_ms / n_q, 2)},
+        "gemm_by_shape": gemm_detail,
+        "clocks": clocks.summary(),
+        "e2e": e2e,
+        "gpu_launches": gpu_launches,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_full_step()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(fp8, stack, stream, steps, world):
+    """H2D of the step's inputs from pinned host memory, the 24 calls, D2H of
+    the three GEMM outputs, per step; CUDA events around the whole loop."""
+    host_in = [{k: v.cpu().pin_memory() for k, v in t.items()} for t in stack.sets[0]]
+    host_out = [{k: torch.empty(L[k].numel(), dtype=torch.bfloat16).pin_memory() for k in ("y", "dx", "dw")}
+                for L in stack.lin]
+    h2d = sum(v.numel() * 2 for t in host_in for v in t.values())
+    d2h = sum(v.numel() * 2 for t in host_out for v in t.values())
+
+    def one():
+        for li, t in enumerate(host_in):
+            for k, v in t.items():
+                stack.sets[0][li][k].copy_(v, non_blocking=True)
+        stack.step(0, stream)
+        for li, L in enumerate(stack.lin):
+            for k in ("y", "dx", "dw"):
+                host_out[li][k].copy_(L[k], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            one()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(steps):
+            one()
+        e1.record(stream)
+    e1.synchronize()
+    barrier(world)
+    t_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    return {"value": stack.flops * steps * world / (t_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": round(t_ms / steps, 3)}
+
+
+# ------------------------------------------------------- the CPU oracle -----
+
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return 1
+
+
+def oracle_prepare(step_tensors):
+    """Untimed set-up for the oracle legs: bf16 inputs as fp32 arrays, their
+    codes and scales (one delayed step each), so that timed samples of the
+    GEMMs run on the step's real operands."""
+    import oracle
+    prep = []
+    for (_, d_in, d_out), t in zip(W.LINEARS, step_tensors):
+        P = {"d_in": d_in, "d_out": d_out, "f": {}, "q": {}, "s": {}}
+        for r, fmt in (("x", E4M3), ("w", E4M3), ("g", E5M2)):
+            P["f"][r] = t[r].reshape(-1).float().numpy()
+            ring = oracle.DelayedRing()
+            ring.step(P["f"][r], fmt)
+            P["q"][r], _, P["s"][r] = ring.step(P["f"][r], fmt)
+        prep.append(P)
+    return prep
+
+
+def oracle_sample_step(prep, frac=1, blk=1):
+    """One step of the oracle on a sample of the workload: the first 1/frac
+    of every quantize input (a delayed ring step) and, of every GEMM, the
+    leading (M/blk) x (N/blk) block of outputs with full K (the oracle called
+    on the operand slices that block needs). frac = blk = 1 is the whole
+    step. Returns (seconds, GEMM FLOPs computed, elements quantized)."""
+    import oracle
+    T = W.TOKENS
+    flops = elems = 0
+    t0 = time.perf_counter()
+    for P in prep:
+        for r, fmt in (("x", E4M3), ("w", E4M3), ("g", E5M2)):
+            x = P["f"][r]
+            n = x.size if frac == 1 else max(16, x.size // frac)
+            oracle.DelayedRing().step(x[:n], fmt)
+            elems += n
+        d_in, d_out, q, s = P["d_in"], P["d_out"], P["q"], P["s"]
+        xq = q["x"].reshape(T, d_in)
+        wq = q["w"].reshape(d_out, d_in)
+        gq = q["g"].reshape(T, d_out)
+        m, n_out, n_in, m_dw = T // blk, d_out // blk, d_in // blk, d_out // blk
+        # forward NT: rows of x, rows of W
+        oracle.mm(xq[:m].reshape(-1), E4M3, wq[:n_out].reshape(-1), E4M3, s["x"], s["w"], oracle.NT,
+                  m, n_out, d_in)
+        # dX NN: rows of g, columns of W ([K = d_out, N = d_in])
+        oracle.mm(gq[:m].reshape(-1), E5M2, np.ascontiguousarray(wq[:, :n_in]).reshape(-1), E4M3,
+                  s["g"], s["w"], oracle.NN, m, n_in, d_out)
+        # dW TN: columns of g ([K = T, M = d_out]), columns of x ([K = T, N = d_in])
+        oracle.mm(np.ascontiguousarray(gq[:, :m_dw]).reshape(-1), E5M2,
+                  np.ascontiguousarray(xq[:, :n_in]).reshape(-1), E4M3, s["g"], s["x"], oracle.TN,
+                  m_dw, n_in, T)
+        flops += 2 * m * n_out * d_in + 2 * m * n_in * d_out + 2 * m_dw * n_in * T
+    return time.perf_counter() - t0, flops, elems
+
+
+def cpu_baseline_full_step():
+    """The oracle as it stands on one full step of the workload (rank 0)."""
+    prep = oracle_prepare(W.stack_tensors(0))
+    dt, flops, elems = oracle_sample_step(prep)
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": _threads(), "kind": "oracle",
+            "sample": f"one full step: 12 delayed quantizes ({elems / 1e6:.1f} M elements) + 12 fp64 GEMMs "
+                      f"({flops / 1e9:.1f} GFLOP)", "seconds": round(dt, 2)}
+
+
+REF_FRAC, REF_BLK = 256, 16
+
+
+def run_reference(args, world, rank):
+    """The oracle on the host cores; each bench step is a bounded sample of
+    the stack step: 1/256 of every quantize input and a (M/16) x (N/16)
+    output block of every GEMM (1/256 of its FLOPs)."""
+    if rank != 0:
+        return
+    prep = oracle_prepare(W.stack_tensors(0))
+    for _ in range(args.warmup):
+        oracle_sample_step(prep, REF_FRAC, REF_BLK)
+    total = flops = 0
+    for _ in range(args.steps):
+        dt, f, _ = oracle_sample_step(prep, REF_FRAC, REF_BLK)
+        total += dt
+        flops += f
+    v = flops / total / 1e12
+    sample = (f"per step: the first 1/{REF_FRAC} of each of the 12 quantize inputs and a (M/{REF_BLK}) x "
+              f"(N/{REF_BLK}) output block, full K, of each of the 12 GEMMs ({flops / args.steps / 1e9:.3f} GFLOP)")
+    line = {"metric": METRIC, "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle: fp32 quantize, fp64 GEMM)",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD, "sample": sample},
+            "cpu_baseline": {"value": round(v, 6), "unit": "TFLOP/s", "cores": _threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_kernel(args):
+    """Single-kernel mode (profiling and sweeps): one GEMM shape or one
+    quantize size, repeated; prints per-launch device time and roofline."""
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    hbm, bf16_burst, _, src = _peaks()
+    st = torch.cuda.Stream()
+    reps = max(args.steps, 1)
+    if args.kernel == "gemm":
+        M, N, K = (int(v) for v in args.shape.split("x"))
+        layout = {"NT": NT, "NN": NN, "TN": TN}[args.layout]
+        sets = []
+        for i in range(2):
+            a = W.fp8_codes((M * K,), E4M3, 9100 + i).cuda()
+            b = W.fp8_codes((N * K,), E4M3, 9200 + i).cuda()
+            sets.append((a, b))
+        sa = torch.ones(1, device="cuda")
+        out = torch.empty(M * N, dtype=torch.bfloat16, device="cuda")
+        call = lambda i: fp8.fp8_mm(sets[i % 2][0], E4M3, sets[i % 2][1], E4M3, sa, sa, layout, M, N, K, 1, 0, 0, 0,
+                                    None, None, 0, out, stream=st)
+        units = 2.0 * M * N * K
+    else:
+        n = int(args.shape)
+        xs = [W.bf16_normal((n,), 1.0, 9300 + i).cuda() for i in range(2)]
+        q = torch.empty(n, dtype=torch.uint8, device="cuda")
+        ring = torch.empty(20, dtype=torch.int32, device="cuda")
+        fp8.fp8_ring_init(ring, 1.0)
+        sc = torch.empty(1, device="cuda")
+        am = torch.empty(1, device="cuda")
+        call = lambda i: fp8.fp8_quantize(xs[i % 2], n, E4M3, ring, q, am, sc, stream=st)
+        units = 3.0 * n
+    with torch.cuda.stream(st):
+        for i in range(max(args.warmup, 3)):
+            call(i)
+    torch.cuda.synchronize()
+    hold_stream(st)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(st):
+        e0.record(st)
+        for i in range(reps):
+            call(i)
+        e1.record(st)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / reps
+    if args.kernel == "gemm":
+        ach = units / (us * 1e-6) / 1e12
+        peak = 2 * bf16_burst
+        print(json.dumps({"kernel": "gemm", "shape": args.shape, "layout": args.layout, "us": round(us, 2),
+                          "tflops": round(ach, 1), "frac_fp8_peak": round(ach / peak, 4), "peak": peak,
+                          "peak_source": src}))
+    else:
+        ach = units / (us * 1e-6) / 1e9
+        print(json.dumps({"kernel": "quantize", "n": int(args.shape), "us": round(us, 2), "gbs": round(ach, 1),
+                          "frac_hbm": round(ach / hbm, 4), "peak": hbm, "peak_source": src}))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--breakdown-reps", type=int, default=20)
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--kernel", choices=["gemm", "quantize"], help="single-kernel mode")
+    ap.add_argument("--shape", default="8192x8192x8192", help="MxNxK for gemm, n for quantize")
+    ap.add_argument("--layout", default="NT", choices=["NT", "NN", "TN"])
+    args = ap.parse_args()
+    if args.kernel:
+        run_kernel(args)
+        return
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank)
+        return
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

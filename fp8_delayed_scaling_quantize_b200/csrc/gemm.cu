@@ -105,19 +105,25 @@ struct Smem {
     static constexpr int kABytes = BM * BK;
     static constexpr int kBBytes = BN * BK;
     static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kBarOffset = STAGES * kStageBytes;
+    static constexpr int kBiasOffset = STAGES * kStageBytes;      // BN fp32 bias values
+    static constexpr int kBarOffset = kBiasOffset + BN * 4;
     // full[S], empty[S], tmem_full[2], tmem_empty[2], then the TMEM slot
     static constexpr int kBytes = kBarOffset + (2 * STAGES + 4) * 8 + 16;
     static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024
     static constexpr uint32_t kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;
 };
 
-template <int BN, bool A_MN, bool B_MN, int STAGES>
+__device__ __forceinline__ void epilogue_bar() {
+    // named barrier 1 over the 4 epilogue warps (128 threads)
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+template <int BN, bool A_MN, bool B_MN, int STAGES, bool HAS_BIAS>
 __global__ void __launch_bounds__(kThreads, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const GemmParams p) {
     using L = Smem<BN, A_MN, B_MN, STAGES>;
-    extern __shared__ uint8_t smem_raw[];
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t s_base = smem_addr(smem);
     const uint32_t s_a = s_base;
@@ -127,6 +133,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     const uint32_t bar_tfull = bar_empty + STAGES * 8;
     const uint32_t bar_tempty = bar_tfull + 2 * 8;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBarOffset + (2 * STAGES + 4) * 8);
+    float* s_bias = reinterpret_cast<float*>(smem + L::kBiasOffset);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -152,6 +159,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // The prologue above overlaps the previous kernel's tail; operands,
+    // scales and the output are touched only after it has completed.
+    griddep_wait();
+    griddep_launch();
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer ---
@@ -228,8 +239,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         // ----------------------------------------------------- epilogue ---
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         const int row_in_tile = q * 32 + lane;
+        const int etid = threadIdx.x - 64;  // 0..127 over the epilogue warps
         const float inv = (1.0f / __ldg(p.sa)) * (1.0f / __ldg(p.sb));
-        const float bscale = p.bias_kind == 2 ? __ldg(p.bias_scale) : 1.0f;
+        const float bscale = (HAS_BIAS && p.bias_kind == 2) ? __ldg(p.bias_scale) : 1.0f;
         int it = 0;
         for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++it) {
             const int mb = t % p.m_tiles;
@@ -238,6 +250,24 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             const int b = rest / p.n_tiles;
             const int buf = it & 1;
             const uint32_t acc_phase = (it >> 1) & 1;
+            if (HAS_BIAS) {
+                // the tile's BN bias values, dequantized once into shared memory
+                epilogue_bar();  // the previous tile's readers are done
+                for (int j = etid; j < BN; j += 128) {
+                    const int col = nb * BN + j;
+                    float v = 0.0f;
+                    if (col < p.N) {
+                        if (p.bias_kind == 1) {
+                            v = __uint_as_float(uint32_t(__ldg(static_cast<const uint16_t*>(p.bias) + col)) << 16);
+                        } else {
+                            v = __fdiv_rn(fp8_to_f32(__ldg(static_cast<const uint8_t*>(p.bias) + col), p.bias_fmt),
+                                          bscale);
+                        }
+                    }
+                    s_bias[j] = v;
+                }
+                epilogue_bar();
+            }
             // every lane waits, then the warp agrees (and reconverges) before
             // the warp-collective TMEM loads
             const bool ok = wait_bounded(bar_tfull + 8 * buf, acc_phase);
@@ -255,16 +285,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                 float y[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const int col = col0 + i;
-                    float bias = 0.0f;
-                    if (p.bias_kind != 0 && col < p.N) {
-                        if (p.bias_kind == 1) {
-                            bias = __uint_as_float(uint32_t(__ldg(static_cast<const uint16_t*>(p.bias) + col)) << 16);
-                        } else {
-                            bias = __fdiv_rn(fp8_to_f32(__ldg(static_cast<const uint8_t*>(p.bias) + col), p.bias_fmt),
-                                             bscale);
-                        }
-                    }
+                    const float bias = HAS_BIAS ? s_bias[c * 32 + i] : 0.0f;
                     y[i] = fmaf(__uint_as_float(r[i]), inv, bias);
                 }
                 if (p.vec_store && col0 + 32 <= p.N) {
@@ -359,10 +380,11 @@ struct HostArgs {
     int64_t batch, stride_b;
 };
 
-template <int BN, bool A_MN, bool B_MN, int STAGES>
-fp8_status launch(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, const HostArgs& h, cudaStream_t st) {
+template <int BN, bool A_MN, bool B_MN, int STAGES, bool HAS_BIAS>
+fp8_status launch_one(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, const HostArgs& h,
+                      cudaStream_t st) {
     using L = Smem<BN, A_MN, B_MN, STAGES>;
-    auto kern = fp8_gemm_kernel<BN, A_MN, B_MN, STAGES>;
+    auto kern = fp8_gemm_kernel<BN, A_MN, B_MN, STAGES, HAS_BIAS>;
     static bool attr_set[64] = {false};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8_ERR_CUDA;
@@ -377,8 +399,13 @@ fp8_status launch(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, co
     const int64_t tiles = int64_t(p.m_tiles) * p.n_tiles * h.batch;
     p.total_tiles = int(tiles);
     const int grid = int(tiles < sm_count() ? tiles : sm_count());
-    kern<<<grid, kThreads, L::kAlloc, st>>>(ta, tb, p);
-    return launch_status();
+    return launch_pdl(kern, grid, kThreads, L::kAlloc, st, ta, tb, p);
+}
+
+template <int BN, bool A_MN, bool B_MN, int STAGES>
+fp8_status launch(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, const HostArgs& h, cudaStream_t st) {
+    return p.bias_kind ? launch_one<BN, A_MN, B_MN, STAGES, true>(ta, tb, p, h, st)
+                       : launch_one<BN, A_MN, B_MN, STAGES, false>(ta, tb, p, h, st);
 }
 
 // Tile-width choice: the widest BN that still gives every SM work; MN-major

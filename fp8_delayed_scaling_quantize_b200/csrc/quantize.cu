@@ -74,6 +74,12 @@ __device__ __forceinline__ void amax4(uint32_t w0, uint32_t w1, float& m) {
     m = fmaxf(m, fabsf(bf_hi(w1)));
 }
 
+__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
 // Block-wide max of a non-negative, non-NaN float; result valid in thread 0.
 __device__ __forceinline__ uint32_t block_max_bits(float m) {
     __shared__ uint32_t warp_max[kThreads / 32];
@@ -93,14 +99,26 @@ __global__ void __launch_bounds__(kThreads)
 quantize_kernel(const uint16_t* __restrict__ x, int64_t n, uint8_t* __restrict__ out8,
                 fp8_ring* ring, uint32_t* amax_acc, float* amax_out, float* scale_out) {
     const float fmax = fmt_max(FMT);
-    float s = 1.0f;
-    if (MODE == kDelayed) {
-        s = *reinterpret_cast<volatile float*>(&ring->scale);
-    } else if (MODE == kCurrentQuant) {
-        const float a = __uint_as_float(*reinterpret_cast<volatile uint32_t*>(amax_acc));
-        s = (a > 0.0f && isfinite(a)) ? scale_from_amax(fmax, a) : 1.0f;
+    griddep_wait();  // inputs and the ring come from earlier kernels
+    // One thread per block reads the scale (or the amax it comes from) and
+    // shares it: thousands of warps loading one address would queue on a
+    // single L2 line.
+    __shared__ float s_scale;
+    if (MODE != kAmaxOnly) {
+        if (threadIdx.x == 0) {
+            float v;
+            if (MODE == kDelayed) {
+                v = *reinterpret_cast<volatile float*>(&ring->scale);
+            } else {
+                const float a = __uint_as_float(*reinterpret_cast<volatile uint32_t*>(amax_acc));
+                v = (a > 0.0f && isfinite(a)) ? scale_from_amax(fmax, a) : 1.0f;
+            }
+            s_scale = v;
+            if (blockIdx.x == 0) *scale_out = v;
+        }
+        __syncthreads();
     }
-    if (MODE != kAmaxOnly && blockIdx.x == 0 && threadIdx.x == 0) *scale_out = s;
+    const float s = MODE == kAmaxOnly ? 1.0f : s_scale;
 
     const uint4* xv = reinterpret_cast<const uint4*>(x);
     uint2* ov = reinterpret_cast<uint2*>(out8);
@@ -132,6 +150,7 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t n, uint8_t* __restrict__
             }
         }
     }
+    griddep_launch();  // the next kernel may start its prologue
     // ragged tail (n mod 8 elements): one thread, scalar
     if (tid == 0) {
         for (int64_t i = units << 3; i < n; ++i) {
@@ -147,12 +166,11 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t n, uint8_t* __restrict__
     if (bits != 0u) atomicMax(acc, bits);
     if (MODE != kDelayed) return;
 
-    // Last-block election: every block publishes its amax, fences, and takes a
-    // ticket; the block holding the final ticket sees every block's amax.
-    __threadfence();
-    const uint32_t ticket = atomicAdd(&ring->ticket, 1u);
+    // Last-block election: every block publishes its amax, then takes a
+    // ticket with acquire-release semantics (its amax is visible before the
+    // ticket moves); the block holding the final ticket sees every amax.
+    const uint32_t ticket = atom_add_acq_rel(&ring->ticket, 1u);
     if (ticket != gridDim.x - 1) return;
-    __threadfence();
     const float a = __uint_as_float(atomicExch(&ring->amax_bits, 0u));
     volatile fp8_ring* r = ring;
     const uint32_t idx = r->idx & (FP8_RING_HISTORY - 1);
@@ -163,11 +181,11 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t n, uint8_t* __restrict__
     if (wmax > 0.0f && isfinite(wmax)) r->scale = scale_from_amax(fmax, wmax);
     r->idx = (idx + 1) & (FP8_RING_HISTORY - 1);
     if (amax_out) *amax_out = a;
-    __threadfence();
-    atomicExch(&ring->ticket, 0u);
+    r->ticket = 0u;  // ready for the next call (visible at the kernel boundary)
 }
 
 __global__ void ring_write_kernel(fp8_ring* ring, fp8_ring value) {
+    griddep_wait();
     const int t = threadIdx.x;
     if (t < FP8_RING_HISTORY) ring->hist[t] = value.hist[t];
     if (t == 0) {
@@ -202,18 +220,16 @@ template <int FMT>
 fp8_status launch_quantize(const uint16_t* x, int64_t n, fp8_ring* ring, uint8_t* out8,
                            float* amax_out, float* scale_out, cudaStream_t st) {
     const int grid = grid_for(n);
-    if (ring) {
-        quantize_kernel<FMT, kDelayed><<<grid, kThreads, 0, st>>>(x, n, out8, ring, nullptr, amax_out,
-                                                                 scale_out);
-        return launch_status();
-    }
+    if (ring)
+        return launch_pdl(quantize_kernel<FMT, kDelayed>, grid, kThreads, 0, st, x, n, out8, ring,
+                          (uint32_t*)nullptr, amax_out, scale_out);
     uint32_t* acc = reinterpret_cast<uint32_t*>(amax_out);
     if (cudaMemsetAsync(acc, 0, sizeof(uint32_t), st) != cudaSuccess) return FP8_ERR_CUDA;
-    quantize_kernel<FMT, kAmaxOnly><<<grid, kThreads, 0, st>>>(x, n, out8, nullptr, acc, nullptr, nullptr);
-    if (launch_status() != FP8_OK) return FP8_ERR_CUDA;
-    quantize_kernel<FMT, kCurrentQuant><<<grid, kThreads, 0, st>>>(x, n, out8, nullptr, acc, nullptr,
-                                                                  scale_out);
-    return launch_status();
+    if (launch_pdl(quantize_kernel<FMT, kAmaxOnly>, grid, kThreads, 0, st, x, n, out8, (fp8_ring*)nullptr, acc,
+                   (float*)nullptr, (float*)nullptr) != FP8_OK)
+        return FP8_ERR_CUDA;
+    return launch_pdl(quantize_kernel<FMT, kCurrentQuant>, grid, kThreads, 0, st, x, n, out8, (fp8_ring*)nullptr,
+                      acc, (float*)nullptr, scale_out);
 }
 
 bool scale_ok(float s) { return s > 0.0f && s <= 3.402823466e38f; }
