@@ -73,6 +73,12 @@ def barrier(world):
         torch.distributed.barrier()
 
 
+def weak_scaling_value(flops_per_step, steps, world, t_ms_max):
+    """Whole-job TFLOP/s: every rank runs `steps` steps of its own replica;
+    the job takes the slowest rank's time."""
+    return flops_per_step * steps * world / (t_ms_max * 1e-3) / 1e12
+
+
 def max_over_ranks(v, world):
     if world == 1:
         return v
@@ -270,7 +276,7 @@ def run_ours(args, world, rank, local):
     barrier(world)
     t_ms = max_over_ranks(e0.elapsed_time(e1), world)
     ms_step = t_ms / args.steps
-    value = stack.flops * args.steps * world / (t_ms * 1e-3) / 1e12
+    value = weak_scaling_value(stack.flops, args.steps, world, t_ms)
 
     # ---- per-kernel breakdown -----------------------------------------
     # Each of the step's 24 launches is repeated back to back between one
@@ -386,7 +392,7 @@ def run_e2e(fp8, stack, stream, steps, world):
     e1.synchronize()
     barrier(world)
     t_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    return {"value": stack.flops * steps * world / (t_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+    return {"value": weak_scaling_value(stack.flops, steps, world, t_ms), "unit": "TFLOP/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": round(t_ms / steps, 3)}
 

@@ -68,6 +68,7 @@ struct GemmParams {
     uint16_t* out;
     int64_t stride_c;
     int vec_store;  // 16-byte stores allowed (N, stride_c multiples of 8, base aligned)
+    int tma_store;  // tiles leave through shared memory and TMA stores (same conditions)
 };
 
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity) {
@@ -105,7 +106,10 @@ struct Smem {
     static constexpr int kABytes = BM * BK;
     static constexpr int kBBytes = BN * BK;
     static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kBiasOffset = STAGES * kStageBytes;      // BN fp32 bias values
+    // per epilogue warp, two 32x32 bf16 staging buffers (64-byte swizzle)
+    static constexpr int kStgBufBytes = 32 * 32 * 2;
+    static constexpr int kStgOffset = STAGES * kStageBytes;
+    static constexpr int kBiasOffset = kStgOffset + 4 * 2 * kStgBufBytes;  // BN fp32 bias values
     static constexpr int kBarOffset = kBiasOffset + BN * 4;
     // full[S], empty[S], tmem_full[2], tmem_empty[2], then the TMEM slot
     static constexpr int kBytes = kBarOffset + (2 * STAGES + 4) * 8 + 16;
@@ -121,7 +125,7 @@ __device__ __forceinline__ void epilogue_bar() {
 template <int BN, bool A_MN, bool B_MN, int STAGES, bool HAS_BIAS>
 __global__ void __launch_bounds__(kThreads, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                const GemmParams p) {
+                const __grid_constant__ CUtensorMap tm_c, const GemmParams p) {
     using L = Smem<BN, A_MN, B_MN, STAGES>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -150,6 +154,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         fence_mbar_init();
         tma_prefetch(&tm_a);
         tma_prefetch(&tm_b);
+        if (p.tma_store) tma_prefetch(&tm_c);
     }
     if (warp == 1) {
         tmem_alloc(smem_addr(tmem_slot), L::kTmemCols);
@@ -242,6 +247,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         const int etid = threadIdx.x - 64;  // 0..127 over the epilogue warps
         const float inv = (1.0f / __ldg(p.sa)) * (1.0f / __ldg(p.sb));
         const float bscale = (HAS_BIAS && p.bias_kind == 2) ? __ldg(p.bias_scale) : 1.0f;
+        const uint32_t s_stg = s_base + L::kStgOffset;
+        int stg_n = 0;  // TMA stores issued by this warp
+        bool failed = false;
         int it = 0;
         for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++it) {
             const int mb = t % p.m_tiles;
@@ -269,9 +277,14 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                 epilogue_bar();
             }
             // every lane waits, then the warp agrees (and reconverges) before
-            // the warp-collective TMEM loads
-            const bool ok = wait_bounded(bar_tfull + 8 * buf, acc_phase);
-            if (!__all_sync(0xffffffffu, ok)) break;
+            // the warp-collective TMEM loads. After a wait gave up, the warp
+            // keeps walking the tiles without waiting so that the epilogue
+            // warps still meet at every named barrier above.
+            if (!failed) {
+                const bool ok = wait_bounded(bar_tfull + 8 * buf, acc_phase);
+                failed = !__all_sync(0xffffffffu, ok);
+            }
+            if (failed) continue;
             tc_fence_after();
             const int row = mb * BM + row_in_tile;
             uint16_t* orow = p.out + int64_t(b) * p.stride_c + int64_t(row) * p.N;
@@ -281,14 +294,43 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                 tmem_ld32(tmem_base + (uint32_t(q * 32) << 16) + buf * BN + c * 32, r);
                 tmem_ld_wait();
                 const int col0 = nb * BN + c * 32;
-                if (row >= p.M || col0 >= p.N) continue;
+                if (col0 >= p.N) continue;                       // warp-uniform
+                if (!p.tma_store && row >= p.M) continue;
                 float y[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const float bias = HAS_BIAS ? s_bias[c * 32 + i] : 0.0f;
                     y[i] = fmaf(__uint_as_float(r[i]), inv, bias);
                 }
-                if (p.vec_store && col0 + 32 <= p.N) {
+                if (p.tma_store) {
+                    // stage the warp's 32 x 32 bf16 block (64-byte swizzle: the
+                    // 16-byte chunk index XOR (row / 2) mod 4 keeps the 8 lanes of
+                    // a store phase on distinct banks), then one TMA store; it
+                    // clips the M / N tails of the output
+                    const uint32_t stg = s_stg + (q * 2 + (stg_n & 1)) * L::kStgBufBytes;
+                    if (stg_n >= 2) {
+                        if (lane == 0) bulk_wait_read<1>();
+                        __syncwarp();
+                    }
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint32_t w0 = pack_bf16x2(y[8 * j + 0], y[8 * j + 1]);
+                        const uint32_t w1 = pack_bf16x2(y[8 * j + 2], y[8 * j + 3]);
+                        const uint32_t w2 = pack_bf16x2(y[8 * j + 4], y[8 * j + 5]);
+                        const uint32_t w3 = pack_bf16x2(y[8 * j + 6], y[8 * j + 7]);
+                        const uint32_t addr = stg + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4);
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w0), "r"(w1),
+                                     "r"(w2), "r"(w3)
+                                     : "memory");
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_3d(&tm_c, stg, col0, mb * BM + q * 32, b);
+                        bulk_commit();
+                    }
+                    ++stg_n;
+                } else if (p.vec_store && col0 + 32 <= p.N) {
                     uint4* dst = reinterpret_cast<uint4*>(orow + col0);
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
@@ -311,6 +353,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             tc_fence_before();
             mbar_arrive(bar_tempty + 8 * buf);
         }
+        // the staging buffers must outlive the stores that read them, and the
+        // output must be complete when the grid is
+        if (p.tma_store && lane == 0) bulk_wait_all();
     }
 
     tc_fence_before();
@@ -362,6 +407,24 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D map over the bf16 output (N, M, batch), 32 x 32 boxes with a 64-byte
+// swizzle matching the epilogue's staging layout.
+bool make_out_map(CUtensorMap* map, void* base, uint64_t n, uint64_t m, uint64_t batch, uint64_t batch_stride_bytes) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    if (batch <= 1 || batch_stride_bytes == 0) {
+        batch = 1;
+        batch_stride_bytes = ((n * m * 2 + 15) / 16) * 16;
+    }
+    cuuint64_t dims[3] = {n, m, batch};
+    cuuint64_t strides[2] = {n * 2, batch_stride_bytes};
+    cuuint32_t box[3] = {32, 32, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
 int sm_count() {
     static int cached[64] = {0};
     int dev = 0;
@@ -381,8 +444,8 @@ struct HostArgs {
 };
 
 template <int BN, bool A_MN, bool B_MN, int STAGES, bool HAS_BIAS>
-fp8_status launch_one(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, const HostArgs& h,
-                      cudaStream_t st) {
+fp8_status launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, GemmParams p,
+                      const HostArgs& h, cudaStream_t st) {
     using L = Smem<BN, A_MN, B_MN, STAGES>;
     auto kern = fp8_gemm_kernel<BN, A_MN, B_MN, STAGES, HAS_BIAS>;
     static bool attr_set[64] = {false};
@@ -399,13 +462,15 @@ fp8_status launch_one(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p
     const int64_t tiles = int64_t(p.m_tiles) * p.n_tiles * h.batch;
     p.total_tiles = int(tiles);
     const int grid = int(tiles < sm_count() ? tiles : sm_count());
-    return launch_pdl(kern, grid, kThreads, L::kAlloc, st, ta, tb, p);
+    return launch_pdl(kern, grid, kThreads, L::kAlloc, st, ta, tb, tc, p);
 }
 
 template <int BN, bool A_MN, bool B_MN, int STAGES>
 fp8_status launch(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, const HostArgs& h, cudaStream_t st) {
-    return p.bias_kind ? launch_one<BN, A_MN, B_MN, STAGES, true>(ta, tb, p, h, st)
-                       : launch_one<BN, A_MN, B_MN, STAGES, false>(ta, tb, p, h, st);
+    CUtensorMap tc = {};
+    if (p.tma_store && !make_out_map(&tc, p.out, p.N, p.M, h.batch, uint64_t(p.stride_c) * 2)) return FP8_ERR_CUDA;
+    return p.bias_kind ? launch_one<BN, A_MN, B_MN, STAGES, true>(ta, tb, tc, p, h, st)
+                       : launch_one<BN, A_MN, B_MN, STAGES, false>(ta, tb, tc, p, h, st);
 }
 
 // Tile-width choice: the widest BN that still gives every SM work; MN-major
@@ -479,6 +544,7 @@ extern "C" fp8_status fp8_mm(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8, f
     p.out = static_cast<uint16_t*>(out);
     p.stride_c = stride_c;
     p.vec_store = (N % 8 == 0) && (stride_c % 8 == 0) && aligned(out, 16);
+    p.tma_store = p.vec_store;
 
     CUtensorMap ta;
     bool ok = a_mn ? make_map(&ta, a8, M, K, batch, uint64_t(stride_a), 128, BK)
