@@ -101,11 +101,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return r;
 }
 
-template <int BN, bool A_MN, bool B_MN, int STAGES>
+// Shared-memory plan of one CTA. CTAS = 2: an MMA pair, each CTA holding its
+// 128 rows of A and BN/2 columns of B per stage.
+template <int BN, int STAGES, int CTAS>
 struct Smem {
     static constexpr int kABytes = BM * BK;
-    static constexpr int kBBytes = BN * BK;
+    static constexpr int kBBytes = (BN / CTAS) * BK;
     static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kStageTx = CTAS * kStageBytes;  // bytes landing on the leader's full barrier
     // per epilogue warp, two 32x32 bf16 staging buffers (64-byte swizzle)
     static constexpr int kStgBufBytes = 32 * 32 * 2;
     static constexpr int kStgOffset = STAGES * kStageBytes;
@@ -122,11 +125,17 @@ __device__ __forceinline__ void epilogue_bar() {
     asm volatile("bar.sync 1, 128;" ::: "memory");
 }
 
-template <int BN, bool A_MN, bool B_MN, int STAGES, bool HAS_BIAS>
+// One kernel for both tile shapes: CTAS = 1 computes 128 x BN tiles per CTA;
+// CTAS = 2 runs as clusters of two CTAs on two SMs computing 256 x BN tiles
+// with tcgen05 cta_group::2 -- the leader issues the MMAs, each CTA loads its
+// own 128 rows of A and BN/2 columns of B (halving each SM's operand
+// traffic) and writes its own 128 output rows.
+template <int BN, bool A_MN, bool B_MN, int STAGES, bool HAS_BIAS, int CTAS>
 __global__ void __launch_bounds__(kThreads, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const __grid_constant__ CUtensorMap tm_c, const GemmParams p) {
-    using L = Smem<BN, A_MN, B_MN, STAGES>;
+    using L = Smem<BN, STAGES, CTAS>;
+    static_assert(!(B_MN && CTAS == 2 && BN != 256), "MN-major B halves must be whole 128-byte atoms");
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t s_base = smem_addr(smem);
@@ -141,6 +150,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const uint32_t rank = CTAS == 2 ? cluster_ctarank() : 0u;  // 0 = the pair's leader
+    const bool leader = rank == 0;
+    const int unit0 = blockIdx.x / CTAS;     // this CTA's first tile (a pair shares it)
+    const int unit_step = gridDim.x / CTAS;  // tiles advance by the number of CTAs (pairs)
 
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -149,7 +162,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar_tfull + 8 * b, 1);
-            mbar_init(bar_tempty + 8 * b, 4 * 32);
+            mbar_init(bar_tempty + 8 * b, CTAS * 4 * 32);
         }
         fence_mbar_init();
         tma_prefetch(&tm_a);
@@ -157,11 +170,12 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         if (p.tma_store) tma_prefetch(&tm_c);
     }
     if (warp == 1) {
-        tmem_alloc(smem_addr(tmem_slot), L::kTmemCols);
-        tmem_relinquish();
+        tmem_alloc<CTAS>(smem_addr(tmem_slot), L::kTmemCols);
+        tmem_relinquish<CTAS>();
     }
     tc_fence_before();
     __syncthreads();
+    if (CTAS == 2) cluster_sync();  // both CTAs' barriers exist before any remote arrive
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     // The prologue above overlaps the previous kernel's tail; operands,
@@ -175,27 +189,37 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < p.total_tiles && ok; t += gridDim.x) {
+            for (int t = unit0; t < p.total_tiles && ok; t += unit_step) {
                 const int mb = t % p.m_tiles;
                 const int rest = t / p.m_tiles;
                 const int nb = rest % p.n_tiles;
                 const int b = rest / p.n_tiles;
                 const int ba = p.a_bcast ? 0 : b;
                 const int bb = p.b_bcast ? 0 : b;
+                const int m0 = mb * BM * CTAS + int(rank) * BM;
+                const int n0 = nb * BN + int(rank) * (BN / CTAS);
                 for (int kb = 0; kb < p.k_blocks; ++kb) {
                     if (!wait_bounded(bar_empty + 8 * stage, phase ^ 1)) { ok = false; break; }
                     const uint32_t full = bar_full + 8 * stage;
-                    mbar_arrive_expect_tx(full, L::kStageBytes);
+                    if (leader) mbar_arrive_expect_tx(full, L::kStageTx);
                     const uint32_t da = s_a + stage * L::kABytes;
                     const uint32_t db = s_b + stage * L::kBBytes;
-                    if (A_MN) tma_load_3d(da, &tm_a, full, mb * BM, kb * BK, ba);
-                    else      tma_load_3d(da, &tm_a, full, kb * BK, mb * BM, ba);
-                    if (B_MN) {
+                    if (CTAS == 1) {
+                        if (A_MN) tma_load_3d(da, &tm_a, full, m0, kb * BK, ba);
+                        else      tma_load_3d(da, &tm_a, full, kb * BK, m0, ba);
+                        if (B_MN) {
 #pragma unroll
-                        for (int h = 0; h < BN / 128; ++h)
-                            tma_load_3d(db + h * 128 * BK, &tm_b, full, nb * BN + h * 128, kb * BK, bb);
+                            for (int h = 0; h < BN / 128; ++h)
+                                tma_load_3d(db + h * 128 * BK, &tm_b, full, n0 + h * 128, kb * BK, bb);
+                        } else {
+                            tma_load_3d(db, &tm_b, full, kb * BK, n0, bb);
+                        }
                     } else {
-                        tma_load_3d(db, &tm_b, full, kb * BK, nb * BN, bb);
+                        const uint32_t lfull = map_to_rank(full, 0);  // the leader's barrier
+                        if (A_MN) tma_load_3d_pair(da, &tm_a, lfull, m0, kb * BK, ba);
+                        else      tma_load_3d_pair(da, &tm_a, lfull, kb * BK, m0, ba);
+                        if (B_MN) tma_load_3d_pair(db, &tm_b, lfull, n0, kb * BK, bb);
+                        else      tma_load_3d_pair(db, &tm_b, lfull, kb * BK, n0, bb);
                     }
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
@@ -208,12 +232,12 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         }
     } else if (warp == 1) {
         // --------------------------------------------------- MMA issuer ---
-        if (lane == 0) {
+        if (lane == 0 && leader) {
             int stage = 0;
             uint32_t phase = 0;
             int it = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < p.total_tiles && ok; t += gridDim.x, ++it) {
+            for (int t = unit0; t < p.total_tiles && ok; t += unit_step, ++it) {
                 const int buf = it & 1;
                 const uint32_t acc_phase = (it >> 1) & 1;
                 if (!wait_bounded(bar_tempty + 8 * buf, acc_phase ^ 1)) break;
@@ -232,12 +256,15 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                                                     : smem_desc_sw128(da + j * 32, 16, 1024);
                         const uint64_t bdesc = B_MN ? smem_desc_sw128(db + j * 32 * 128, 128 * BK, 1024)
                                                     : smem_desc_sw128(db + j * 32, 16, 1024);
-                        mma_f8f6f4(d_tmem, adesc, bdesc, p.idesc, (kb | j) != 0);
+                        mma_f8f6f4<CTAS>(d_tmem, adesc, bdesc, p.idesc, (kb | j) != 0);
                     }
-                    mma_commit(bar_empty + 8 * stage);
+                    // release the stage (in both CTAs of a pair)
+                    if (CTAS == 1) mma_commit(bar_empty + 8 * stage);
+                    else           mma_commit_pair(bar_empty + 8 * stage);
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
-                mma_commit(bar_tfull + 8 * buf);
+                if (CTAS == 1) mma_commit(bar_tfull + 8 * buf);
+                else           mma_commit_pair(bar_tfull + 8 * buf);
             }
         }
     } else {
@@ -251,13 +278,14 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         int stg_n = 0;  // TMA stores issued by this warp
         bool failed = false;
         int it = 0;
-        for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++it) {
+        for (int t = unit0; t < p.total_tiles; t += unit_step, ++it) {
             const int mb = t % p.m_tiles;
             const int rest = t / p.m_tiles;
             const int nb = rest % p.n_tiles;
             const int b = rest / p.n_tiles;
             const int buf = it & 1;
             const uint32_t acc_phase = (it >> 1) & 1;
+            const int m0 = mb * BM * CTAS + int(rank) * BM;  // this CTA's first output row
             if (HAS_BIAS) {
                 // the tile's BN bias values, dequantized once into shared memory
                 epilogue_bar();  // the previous tile's readers are done
@@ -286,7 +314,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             }
             if (failed) continue;
             tc_fence_after();
-            const int row = mb * BM + row_in_tile;
+            const int row = m0 + row_in_tile;
             uint16_t* orow = p.out + int64_t(b) * p.stride_c + int64_t(row) * p.N;
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
@@ -326,7 +354,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        tma_store_3d(&tm_c, stg, col0, mb * BM + q * 32, b);
+                        tma_store_3d(&tm_c, stg, col0, m0 + q * 32, b);
                         bulk_commit();
                     }
                     ++stg_n;
@@ -351,7 +379,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                 }
             }
             tc_fence_before();
-            mbar_arrive(bar_tempty + 8 * buf);
+            // release the accumulator to the MMA issuer (the pair's leader)
+            if (CTAS == 1) mbar_arrive(bar_tempty + 8 * buf);
+            else           mbar_arrive_cluster(map_to_rank(bar_tempty + 8 * buf, 0));
         }
         // the staging buffers must outlive the stores that read them, and the
         // output must be complete when the grid is
@@ -360,10 +390,11 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
 
     tc_fence_before();
     __syncthreads();
+    if (CTAS == 2) cluster_sync();  // neither CTA leaves while the other may still signal it
     tc_fence_after();
     if (warp == 1) {
         __syncwarp();
-        tmem_dealloc(tmem_base, L::kTmemCols);
+        tmem_dealloc<CTAS>(tmem_base, L::kTmemCols);
     }
 }
 
@@ -443,11 +474,11 @@ struct HostArgs {
     int64_t batch, stride_b;
 };
 
-template <int BN, bool A_MN, bool B_MN, int STAGES, bool HAS_BIAS>
+template <int BN, bool A_MN, bool B_MN, int STAGES, bool HAS_BIAS, int CTAS>
 fp8_status launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, GemmParams p,
                       const HostArgs& h, cudaStream_t st) {
-    using L = Smem<BN, A_MN, B_MN, STAGES>;
-    auto kern = fp8_gemm_kernel<BN, A_MN, B_MN, STAGES, HAS_BIAS>;
+    using L = Smem<BN, STAGES, CTAS>;
+    auto kern = fp8_gemm_kernel<BN, A_MN, B_MN, STAGES, HAS_BIAS, CTAS>;
     static bool attr_set[64] = {false};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8_ERR_CUDA;
@@ -456,40 +487,49 @@ fp8_status launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
             return FP8_ERR_CUDA;
         attr_set[dev] = true;
     }
-    p.idesc = sm100::instr_desc_f8(h.fa, h.fb, A_MN ? 1 : 0, B_MN ? 1 : 0, BM, BN);
-    p.m_tiles = (p.M + BM - 1) / BM;
+    p.idesc = sm100::instr_desc_f8(h.fa, h.fb, A_MN ? 1 : 0, B_MN ? 1 : 0, BM * CTAS, BN);
+    p.m_tiles = (p.M + BM * CTAS - 1) / (BM * CTAS);
     p.n_tiles = (p.N + BN - 1) / BN;
     const int64_t tiles = int64_t(p.m_tiles) * p.n_tiles * h.batch;
     p.total_tiles = int(tiles);
-    const int grid = int(tiles < sm_count() ? tiles : sm_count());
-    return launch_pdl(kern, grid, kThreads, L::kAlloc, st, ta, tb, tc, p);
+    const int64_t units_max = sm_count() / CTAS;
+    const int units = int(tiles < units_max ? tiles : units_max);
+    return launch_pdl(kern, units * CTAS, kThreads, L::kAlloc, st, CTAS, ta, tb, tc, p);
 }
 
-template <int BN, bool A_MN, bool B_MN, int STAGES>
+template <int BN, bool A_MN, bool B_MN, int STAGES, int CTAS>
 fp8_status launch(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, const HostArgs& h, cudaStream_t st) {
     CUtensorMap tc = {};
     if (p.tma_store && !make_out_map(&tc, p.out, p.N, p.M, h.batch, uint64_t(p.stride_c) * 2)) return FP8_ERR_CUDA;
-    return p.bias_kind ? launch_one<BN, A_MN, B_MN, STAGES, true>(ta, tb, tc, p, h, st)
-                       : launch_one<BN, A_MN, B_MN, STAGES, false>(ta, tb, tc, p, h, st);
+    return p.bias_kind ? launch_one<BN, A_MN, B_MN, STAGES, true, CTAS>(ta, tb, tc, p, h, st)
+                       : launch_one<BN, A_MN, B_MN, STAGES, false, CTAS>(ta, tb, tc, p, h, st);
 }
 
-// Tile-width choice: the widest BN that still gives every SM work; MN-major
-// B needs BN >= 128 (the tile is whole 128-byte swizzle atoms along N).
+// Tile choice for 148 SMs. Large problems (at least two waves of 256 x 256
+// tiles) run on SM pairs (cta_group::2), which halves each SM's operand
+// traffic; otherwise the widest 1-SM tile that still gives every SM work.
+// MN-major B needs whole 128-byte swizzle atoms along N per CTA.
 template <bool A_MN, bool B_MN>
 fp8_status dispatch(const CUtensorMap& ta, GemmParams p, const HostArgs& h, cudaStream_t st) {
-    const int64_t m_tiles = (p.M + BM - 1) / BM;
     const int64_t sms = sm_count();
+    const int64_t m_tiles = (p.M + BM - 1) / BM;
+    const int64_t pair_tiles = ((p.M + 2 * BM - 1) / (2 * BM)) * ((p.N + 255) / 256) * h.batch;
+    const bool pair = p.M > BM && p.N > 128 && pair_tiles >= sms;
     int bn = 256;
-    if (p.N <= 128 || m_tiles * ((p.N + 255) / 256) * h.batch < sms) bn = 128;
-    if (!B_MN && (p.N <= 64 || (bn == 128 && m_tiles * ((p.N + 127) / 128) * h.batch < sms / 2))) bn = 64;
+    if (!pair) {
+        if (p.N <= 128 || m_tiles * ((p.N + 255) / 256) * h.batch < sms) bn = 128;
+        if (!B_MN && (p.N <= 64 || (bn == 128 && m_tiles * ((p.N + 127) / 128) * h.batch < sms / 2))) bn = 64;
+    }
     CUtensorMap tb;
     const uint64_t sb_bytes = uint64_t(h.stride_b);
+    const uint32_t b_box_n = pair ? bn / 2 : bn;  // N extent one CTA loads
     const bool ok = B_MN ? make_map(&tb, h.b8, p.N, p.K, h.batch, sb_bytes, 128, BK)
-                         : make_map(&tb, h.b8, p.K, p.N, h.batch, sb_bytes, BK, bn);
+                         : make_map(&tb, h.b8, p.K, p.N, h.batch, sb_bytes, BK, b_box_n);
     if (!ok) return FP8_ERR_CUDA;
-    if (bn == 256) return launch<256, A_MN, B_MN, 4>(ta, tb, p, h, st);
-    if (bn == 128) return launch<128, A_MN, B_MN, 6>(ta, tb, p, h, st);
-    if constexpr (!B_MN) return launch<64, A_MN, B_MN, 8>(ta, tb, p, h, st);
+    if (pair) return launch<256, A_MN, B_MN, 6, 2>(ta, tb, p, h, st);
+    if (bn == 256) return launch<256, A_MN, B_MN, 4, 1>(ta, tb, p, h, st);
+    if (bn == 128) return launch<128, A_MN, B_MN, 6, 1>(ta, tb, p, h, st);
+    if constexpr (!B_MN) return launch<64, A_MN, B_MN, 8, 1>(ta, tb, p, h, st);
     return FP8_ERR_UNSUPPORTED;
 }
 

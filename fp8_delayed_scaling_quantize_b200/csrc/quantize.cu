@@ -221,14 +221,14 @@ fp8_status launch_quantize(const uint16_t* x, int64_t n, fp8_ring* ring, uint8_t
                            float* amax_out, float* scale_out, cudaStream_t st) {
     const int grid = grid_for(n);
     if (ring)
-        return launch_pdl(quantize_kernel<FMT, kDelayed>, grid, kThreads, 0, st, x, n, out8, ring,
+        return launch_pdl(quantize_kernel<FMT, kDelayed>, grid, kThreads, 0, st, 1, x, n, out8, ring,
                           (uint32_t*)nullptr, amax_out, scale_out);
     uint32_t* acc = reinterpret_cast<uint32_t*>(amax_out);
     if (cudaMemsetAsync(acc, 0, sizeof(uint32_t), st) != cudaSuccess) return FP8_ERR_CUDA;
-    if (launch_pdl(quantize_kernel<FMT, kAmaxOnly>, grid, kThreads, 0, st, x, n, out8, (fp8_ring*)nullptr, acc,
+    if (launch_pdl(quantize_kernel<FMT, kAmaxOnly>, grid, kThreads, 0, st, 1, x, n, out8, (fp8_ring*)nullptr, acc,
                    (float*)nullptr, (float*)nullptr) != FP8_OK)
         return FP8_ERR_CUDA;
-    return launch_pdl(quantize_kernel<FMT, kCurrentQuant>, grid, kThreads, 0, st, x, n, out8, (fp8_ring*)nullptr,
+    return launch_pdl(quantize_kernel<FMT, kCurrentQuant>, grid, kThreads, 0, st, 1, x, n, out8, (fp8_ring*)nullptr,
                       acc, (float*)nullptr, scale_out);
 }
 
