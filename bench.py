@@ -193,27 +193,41 @@ class Stack:
         L = self.lin[li]
         return 2 * W.TOKENS * L["d_in"] * L["d_out"]
 
-    def step(self, s, stream, events=None):
-        """Issue one step on input set s. With `events`, record a CUDA event
-        pair around every launch: events[kind] += [(start, end, units)]."""
+    def step(self, s, stream, side=None):
+        """Issue one training step of the stack on input set s: the forward
+        of every linear in order (quantize x and W, y = x W^T), then the
+        backward in reverse order (quantize g, dX = g W, dW = g^T x).
+
+        With a `side` stream, the work a linear layer can overlap runs on it:
+        W's quantize beside x's, and dW beside dX (both only need g8); the
+        streams fork and join around each pair, so the dependencies between
+        linears are those of a sequential model."""
         fp8 = self.fp8
-        for li in range(len(self.lin)):
-            for args in self.quant_calls(s, li):
-                if events is not None:
-                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    e0.record(stream)
-                fp8.fp8_quantize(*args, stream=stream)
-                if events is not None:
-                    e1.record(stream)
-                    events["quantize"].append((e0, e1, args[1]))
-            for args in self.gemm_calls(li):
-                if events is not None:
-                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    e0.record(stream)
-                fp8.fp8_mm(*args, stream=stream)
-                if events is not None:
-                    e1.record(stream)
-                    events["gemm"].append((e0, e1, self.gemm_flops(li), args[6], args[7:10]))
+        n = len(self.lin)
+        for li in range(n):
+            qx, qw, _ = self.quant_calls(s, li)
+            fwd, _, _ = self.gemm_calls(li)
+            if side is not None:
+                side.wait_stream(stream)
+                fp8.fp8_quantize(*qw, stream=side)
+                fp8.fp8_quantize(*qx, stream=stream)
+                stream.wait_stream(side)
+            else:
+                fp8.fp8_quantize(*qx, stream=stream)
+                fp8.fp8_quantize(*qw, stream=stream)
+            fp8.fp8_mm(*fwd, stream=stream)
+        for li in reversed(range(n)):
+            _, _, qg = self.quant_calls(s, li)
+            _, dx, dw = self.gemm_calls(li)
+            fp8.fp8_quantize(*qg, stream=stream)
+            if side is not None:
+                side.wait_stream(stream)
+                fp8.fp8_mm(*dw, stream=side)
+                fp8.fp8_mm(*dx, stream=stream)
+                stream.wait_stream(side)
+            else:
+                fp8.fp8_mm(*dx, stream=stream)
+                fp8.fp8_mm(*dw, stream=stream)
 
 
 def hold_stream(stream, us=2000):
@@ -236,13 +250,14 @@ def run_ours(args, world, rank, local):
     hbm, bf16_burst, bf16_sust, peak_src = _peaks()
     fp8_burst = 2.0 * bf16_burst      # dense FP8 = 2x dense bf16 (nominal 4.5 / 2.25 PF/s)
     stream = torch.cuda.Stream()
+    side = None if args.one_stream else torch.cuda.Stream()
     stack = Stack(fp8)
     torch.cuda.synchronize()
 
     # warm-up (eager) also sets kernel attributes before any capture
     with torch.cuda.stream(stream):
         for i in range(max(args.warmup, 3)):
-            stack.step(i % N_SETS, stream)
+            stack.step(i % N_SETS, stream, side)
     torch.cuda.synchronize()
 
     graphs = []
@@ -250,7 +265,7 @@ def run_ours(args, world, rank, local):
         for s in range(N_SETS):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
-                stack.step(s, stream)
+                stack.step(s, stream, side)
             graphs.append(g)
         torch.cuda.synchronize()
         for i in range(max(args.warmup, 3)):
@@ -269,7 +284,7 @@ def run_ours(args, world, rank, local):
                 if graphs:
                     graphs[i % N_SETS].replay()
                 else:
-                    stack.step(i % N_SETS, stream)
+                    stack.step(i % N_SETS, stream, side)
             e1.record(stream)
         e1.synchronize()
     torch.cuda.synchronize()
@@ -318,7 +333,7 @@ def run_ours(args, world, rank, local):
     # ---- e2e: host buffers through the public API ------------------------
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(fp8, stack, stream, args.e2e_steps, world)
+        e2e = run_e2e(fp8, stack, stream, args.e2e_steps, world, side)
         e2e["value"] = round(e2e["value"], 3)
 
     gpu_launches = 24 * args.steps
@@ -332,7 +347,9 @@ def run_ours(args, world, rank, local):
                    "gemm_gflop_per_step": round(stack.flops / 1e9, 2),
                    "quant_elems_per_step": stack.q_elems,
                    "l2": f"{N_SETS} rotating input sets ({N_SETS * 2 * stack.q_elems / 1e6:.0f} MB bf16) > 126 MB L2",
-                   "launch": "CUDA graph per step" if graphs else "eager",
+                   "launch": ("CUDA graph per step" if graphs else "eager") +
+                             (", 1 stream" if side is None else ", 2 streams (x||W quantize, dX||dW)"),
+                   "order": "forward over linears, then backward in reverse",
                    "parallelism": f"replicas x{world}"},
         "quantize_gbs": round(quant_gbs, 1),
         "roofline": {"bound": "tensor", "achieved": round(gemm_tf, 1), "peak": round(fp8_burst, 1),
@@ -360,7 +377,7 @@ def run_ours(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
-def run_e2e(fp8, stack, stream, steps, world):
+def run_e2e(fp8, stack, stream, steps, world, side=None):
     """H2D of the step's inputs from pinned host memory, the 24 calls, D2H of
     the three GEMM outputs, per step; CUDA events around the whole loop."""
     host_in = [{k: v.cpu().pin_memory() for k, v in t.items()} for t in stack.sets[0]]
@@ -373,7 +390,7 @@ def run_e2e(fp8, stack, stream, steps, world):
         for li, t in enumerate(host_in):
             for k, v in t.items():
                 stack.sets[0][li][k].copy_(v, non_blocking=True)
-        stack.step(0, stream)
+        stack.step(0, stream, side)
         for li, L in enumerate(stack.lin):
             for k in ("y", "dx", "dw"):
                 host_out[li][k].copy_(L[k], non_blocking=True)
@@ -561,6 +578,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--one-stream", action="store_true", help="issue the whole step on one stream")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--breakdown-reps", type=int, default=20)

@@ -44,7 +44,7 @@ assert ctypes.sizeof(fp8_ring) == FP8_RING_BYTES
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is not built; run `python -m fp8_delayed_scaling_quantize_b200.build`")
+        raise ImportError(f"{LIB_PATH} is not built; run `python fp8_delayed_scaling_quantize_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     P, I64, I, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
     sig = {
@@ -56,9 +56,14 @@ def _load():
         "fp8_quantize": (I, [P, I64, I, P, P, P, P, P]),
         "fp8_mm": (I, [P, I, P, I, P, P, I, I64, I64, I64, I64, I64, I64, I64, P, P, I, P, P]),
         "fp8_last_device_error": (I, []),
+        "fp8_selftest_wait_timeout": (I, [ctypes.c_uint32, P]),
     }
     for name, (res, args) in sig.items():
-        fn = getattr(lib, name)
+        try:
+            fn = getattr(lib, name)
+        except AttributeError:
+            raise ImportError(f"{LIB_PATH} lacks {name}: it is stale; rebuild it with "
+                              f"`python fp8_delayed_scaling_quantize_b200/build.py`") from None
         fn.restype = res
         fn.argtypes = args
     return lib
@@ -127,6 +132,10 @@ def fp8_mm(a8, fa, b8, fb, sa, sb, layout, M, N, K, batch, stride_a, stride_b, s
 
 def fp8_last_device_error():
     return _check(lib.fp8_last_device_error(), "fp8_last_device_error")
+
+
+def fp8_selftest_wait_timeout(limit_us: int, stream=None):
+    return _check(lib.fp8_selftest_wait_timeout(int(limit_us), _stream(stream)), "fp8_selftest_wait_timeout")
 
 
 def raw_status(fn_name: str, *args) -> int:

@@ -2,7 +2,8 @@
 
 Compiles for sm_100a only (B200), with IEEE fp32 semantics: no fast-math,
 no flush-to-zero, round-to-nearest division (the quantize and epilogue
-arithmetic depends on these). Usage: ``python -m fp8_delayed_scaling_quantize_b200.build``.
+arithmetic depends on these). Usage: ``python fp8_delayed_scaling_quantize_b200/build.py``
+(run as a file: importing the package loads the library this script builds).
 """
 
 import os
@@ -14,6 +15,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libfp8lite.so")
 SOURCES = ("quantize.cu", "gemm.cu")
+
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

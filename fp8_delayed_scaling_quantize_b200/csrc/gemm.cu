@@ -71,16 +71,28 @@ struct GemmParams {
     int tma_store;  // tiles leave through shared memory and TMA stores (same conditions)
 };
 
-__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity) {
+// Wait for phase `parity` of the mbarrier at `bar`, giving up after
+// `limit_ns`: then the library's device error word is set and false returned.
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 1023u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+        if ((i & 1023u) == 0 && globaltimer_ns() - t0 > limit_ns) {
             atomicOr(&g_device_error, 1u);
             return false;
         }
     }
+}
+
+// Diagnostic: one thread waits, through the same bounded wait the GEMM
+// uses, on a shared-memory barrier that nothing ever arrives at.
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t b = smem_addr(&bar);
+    mbar_init(b, 1);
+    fence_mbar_init();
+    wait_bounded(b, 0, limit_ns);
 }
 
 // One FP8 code -> fp32 (exact: every E4M3 / E5M2 value is an fp16 value).
@@ -505,21 +517,44 @@ fp8_status launch(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, co
                        : launch_one<BN, A_MN, B_MN, STAGES, false, CTAS>(ta, tb, tc, p, h, st);
 }
 
-// Tile choice for 148 SMs. Large problems (at least two waves of 256 x 256
-// tiles) run on SM pairs (cta_group::2), which halves each SM's operand
-// traffic; otherwise the widest 1-SM tile that still gives every SM work.
-// MN-major B needs whole 128-byte swizzle atoms along N per CTA.
+// Tile choice for 148 SMs by a small cost model: a persistent grid walks
+// ceil(tiles / CTAs) rounds of tiles, each costing k_blocks times the
+// per-k-block time of that tile shape, plus the one epilogue left exposed at
+// the end. The per-k-block times (microseconds at the clocks seen under load)
+// and epilogue times were measured on B200 with this kernel: 128x256 0.48,
+// 128x128 0.40, 128x64 0.30, an SM pair's 256x256 0.43. Pairs are used only
+// with at least one 256x256 tile per SM (below that their coarser grain
+// loses). MN-major B needs whole 128-byte swizzle atoms along N per CTA.
+struct TileChoice {
+    bool pair;
+    int bn;
+};
+
+inline TileChoice choose_tile(int64_t M, int64_t N, int64_t K, int64_t batch, bool b_mn, int64_t sms) {
+    const int64_t kb = (K + BK - 1) / BK;
+    auto cost = [&](int64_t rows, int bn, int64_t units, double t_k, double t_epi) {
+        const int64_t tiles = ((M + rows - 1) / rows) * ((N + bn - 1) / bn) * batch;
+        const int64_t rounds = (tiles + units - 1) / units;
+        return double(rounds) * double(kb) * t_k + t_epi;
+    };
+    const int64_t pair_tiles = ((M + 2 * BM - 1) / (2 * BM)) * ((N + 255) / 256) * batch;
+    if (M > BM && N > 128 && pair_tiles >= sms) return {true, 256};
+    TileChoice best = {false, 256};
+    double best_cost = cost(BM, 256, sms, 0.48, 2.0);
+    const double c128 = cost(BM, 128, sms, 0.40, 1.0);
+    if (c128 < best_cost) { best = {false, 128}; best_cost = c128; }
+    if (!b_mn) {
+        const double c64 = cost(BM, 64, sms, 0.30, 0.5);
+        if (c64 < best_cost) { best = {false, 64}; best_cost = c64; }
+    }
+    return best;
+}
+
 template <bool A_MN, bool B_MN>
 fp8_status dispatch(const CUtensorMap& ta, GemmParams p, const HostArgs& h, cudaStream_t st) {
-    const int64_t sms = sm_count();
-    const int64_t m_tiles = (p.M + BM - 1) / BM;
-    const int64_t pair_tiles = ((p.M + 2 * BM - 1) / (2 * BM)) * ((p.N + 255) / 256) * h.batch;
-    const bool pair = p.M > BM && p.N > 128 && pair_tiles >= sms;
-    int bn = 256;
-    if (!pair) {
-        if (p.N <= 128 || m_tiles * ((p.N + 255) / 256) * h.batch < sms) bn = 128;
-        if (!B_MN && (p.N <= 64 || (bn == 128 && m_tiles * ((p.N + 127) / 128) * h.batch < sms / 2))) bn = 64;
-    }
+    const TileChoice tc = choose_tile(p.M, p.N, p.K, h.batch, B_MN, sm_count());
+    const bool pair = tc.pair;
+    const int bn = tc.bn;
     CUtensorMap tb;
     const uint64_t sb_bytes = uint64_t(h.stride_b);
     const uint32_t b_box_n = pair ? bn / 2 : bn;  // N extent one CTA loads
@@ -606,4 +641,10 @@ extern "C" fp8_status fp8_last_device_error(void) {
     const uint32_t zero = 0;
     if (v != 0 && cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return FP8_ERR_CUDA;
     return v ? FP8_ERR_DEVICE_TIMEOUT : FP8_OK;
+}
+
+extern "C" fp8_status fp8_selftest_wait_timeout(uint32_t limit_us, void* stream) {
+    if (limit_us == 0 || limit_us > 1000000u) return FP8_ERR_INVALID_ARG;
+    selftest_wait_kernel<<<1, 1, 0, as_stream(stream)>>>(uint64_t(limit_us) * 1000ull);
+    return launch_status();
 }

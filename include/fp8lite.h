@@ -175,6 +175,15 @@ FP8LITE_API fp8_status fp8_mm(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8, 
  * FP8_OK otherwise, FP8_ERR_CUDA if the synchronisation failed. */
 FP8LITE_API fp8_status fp8_last_device_error(void);
 
+/* Diagnostic of the failure path: launches one tiny kernel whose single
+ * thread waits, through the same bounded wait the GEMM uses, on a barrier
+ * that nothing arrives at. After limit_us (1 .. 1e6 microseconds) the wait
+ * gives up and records a timeout in the device error word, exactly as a stuck
+ * GEMM would, and the kernel returns normally (no fault, no trap): the next
+ * fp8_last_device_error() reports FP8_ERR_DEVICE_TIMEOUT and clears it.
+ * Errors: FP8_ERR_INVALID_ARG (limit out of range), FP8_ERR_CUDA. */
+FP8LITE_API fp8_status fp8_selftest_wait_timeout(uint32_t limit_us, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

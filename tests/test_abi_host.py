@@ -12,7 +12,11 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def fp8():
-    from fp8_delayed_scaling_quantize_b200 import build
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "fp8lite_build", os.path.join(ROOT, "fp8_delayed_scaling_quantize_b200", "build.py"))
+    build = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(build)
     build.build()
     import fp8_delayed_scaling_quantize_b200 as m
     return m

@@ -1,0 +1,38 @@
+"""Failure detection without a GPU fault: a bounded device wait that runs out
+(a barrier nothing arrives at) is reported through fp8_last_device_error, the
+error word is cleared by reading it, and the context stays usable."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+def test_bounded_wait_times_out_cleanly():
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    import gpu_util as g
+    fp8.fp8_last_device_error()                     # start clean
+    fp8.fp8_selftest_wait_timeout(2000)             # 2 ms limit
+    with pytest.raises(fp8.Fp8Error) as e:
+        fp8.fp8_last_device_error()
+    assert e.value.status == fp8.FP8_ERR_DEVICE_TIMEOUT
+    fp8.fp8_last_device_error()                     # reading cleared it
+    # the context still computes correctly
+    a8 = W.fp8_codes((128 * 128,), 0, 1)
+    b8 = W.fp8_codes((128 * 128,), 0, 2)
+    s = torch.ones(1, device="cuda")
+    out = g.mm(a8.cuda(), 0, b8.cuda(), 0, s, s, fp8.FP8_NT, 128, 128, 128)
+    y, sums = oracle.mm(a8.numpy(), 0, b8.numpy(), 0, 1.0, 1.0, oracle.NT, 128, 128, 128)
+    got = out.float().cpu().numpy().reshape(1, 128, 128)
+    assert np.all(np.abs(got - y) <= oracle.tolerance(y, sums))
+    fp8.fp8_last_device_error()
+
+
+def test_selftest_argument_validation():
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    assert fp8.raw_status("fp8_selftest_wait_timeout", 0, None) == fp8.FP8_ERR_INVALID_ARG
+    assert fp8.raw_status("fp8_selftest_wait_timeout", 2_000_000, None) == fp8.FP8_ERR_INVALID_ARG
