@@ -523,7 +523,21 @@ def run_kernel(args):
     hbm, bf16_burst, _, src = _peaks()
     st = torch.cuda.Stream()
     reps = max(args.steps, 1)
-    if args.kernel == "gemm":
+    if args.kernel == "cublaslt":
+        # in-box comparison: cuBLASLt's FP8 GEMM through torch._scaled_mm on
+        # the same NT problem (A [M,K] row-major, B [N,K] row-major = a
+        # column-major [K,N] operand); scales are its dequantisation factors
+        M, N, K = (int(v) for v in args.shape.split("x"))
+        sets = []
+        for i in range(2):
+            a = W.fp8_codes((M, K), E4M3, 9100 + i).cuda().view(torch.float8_e4m3fn)
+            b = W.fp8_codes((N, K), E4M3, 9200 + i).cuda().view(torch.float8_e4m3fn)
+            sets.append((a, b))
+        one = torch.ones((), device="cuda")
+        call = lambda i: torch._scaled_mm(sets[i % 2][0], sets[i % 2][1].t(), scale_a=one, scale_b=one,
+                                          out_dtype=torch.bfloat16)
+        units = 2.0 * M * N * K
+    elif args.kernel == "gemm":
         M, N, K = (int(v) for v in args.shape.split("x"))
         layout = {"NT": NT, "NN": NN, "TN": TN}[args.layout]
         sets = []
@@ -559,10 +573,11 @@ def run_kernel(args):
         e1.record(st)
     torch.cuda.synchronize()
     us = e0.elapsed_time(e1) * 1e3 / reps
-    if args.kernel == "gemm":
+    if args.kernel in ("gemm", "cublaslt"):
         ach = units / (us * 1e-6) / 1e12
         peak = 2 * bf16_burst
-        print(json.dumps({"kernel": "gemm", "shape": args.shape, "layout": args.layout, "us": round(us, 2),
+        print(json.dumps({"kernel": args.kernel, "shape": args.shape,
+                          "layout": args.layout if args.kernel == "gemm" else "NT", "us": round(us, 2),
                           "tflops": round(ach, 1), "frac_fp8_peak": round(ach / peak, 4), "peak": peak,
                           "peak_source": src}))
     else:
@@ -583,7 +598,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--breakdown-reps", type=int, default=20)
     ap.add_argument("--e2e-steps", type=int, default=10)
-    ap.add_argument("--kernel", choices=["gemm", "quantize"], help="single-kernel mode")
+    ap.add_argument("--kernel", choices=["gemm", "quantize", "cublaslt"], help="single-kernel mode")
     ap.add_argument("--shape", default="8192x8192x8192", help="MxNxK for gemm, n for quantize")
     ap.add_argument("--layout", default="NT", choices=["NT", "NN", "TN"])
     args = ap.parse_args()

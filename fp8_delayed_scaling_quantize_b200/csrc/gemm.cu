@@ -57,6 +57,7 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 struct GemmParams {
     int M, N, K;
     int m_tiles, n_tiles, k_blocks, total_tiles;
+    int group_m;  // tiles are walked in groups of this many M-tile rows
     int a_bcast, b_bcast;
     uint32_t idesc;
     const float* sa;
@@ -132,6 +133,24 @@ struct Smem {
     static constexpr uint32_t kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;
 };
 
+// Tile order: batch outermost; inside a batch, groups of `group_m` M-tile
+// rows, walked M-fastest within the group, then N. A wave of concurrently
+// running tiles then covers a compact block of rows and columns whose A and B
+// panels stay resident in L2 (an M-fastest walk over all rows streams the
+// whole A through L2 every wave).
+__device__ __forceinline__ void tile_coords(int t, const GemmParams& p, int& mb, int& nb, int& b) {
+    const int per_batch = p.m_tiles * p.n_tiles;
+    b = t / per_batch;
+    const int r = t - b * per_batch;
+    const int per_group = p.group_m * p.n_tiles;
+    const int g = r / per_group;
+    const int first_m = g * p.group_m;
+    const int rows = min(p.group_m, p.m_tiles - first_m);
+    const int i = r - g * per_group;
+    mb = first_m + i % rows;
+    nb = i / rows;
+}
+
 __device__ __forceinline__ void epilogue_bar() {
     // named barrier 1 over the 4 epilogue warps (128 threads)
     asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -202,10 +221,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             uint32_t phase = 0;
             bool ok = true;
             for (int t = unit0; t < p.total_tiles && ok; t += unit_step) {
-                const int mb = t % p.m_tiles;
-                const int rest = t / p.m_tiles;
-                const int nb = rest % p.n_tiles;
-                const int b = rest / p.n_tiles;
+                int mb, nb, b;
+                tile_coords(t, p, mb, nb, b);
                 const int ba = p.a_bcast ? 0 : b;
                 const int bb = p.b_bcast ? 0 : b;
                 const int m0 = mb * BM * CTAS + int(rank) * BM;
@@ -291,10 +308,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         bool failed = false;
         int it = 0;
         for (int t = unit0; t < p.total_tiles; t += unit_step, ++it) {
-            const int mb = t % p.m_tiles;
-            const int rest = t / p.m_tiles;
-            const int nb = rest % p.n_tiles;
-            const int b = rest / p.n_tiles;
+            int mb, nb, b;
+            tile_coords(t, p, mb, nb, b);
             const int buf = it & 1;
             const uint32_t acc_phase = (it >> 1) & 1;
             const int m0 = mb * BM * CTAS + int(rank) * BM;  // this CTA's first output row
@@ -504,6 +519,7 @@ fp8_status launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
     p.n_tiles = (p.N + BN - 1) / BN;
     const int64_t tiles = int64_t(p.m_tiles) * p.n_tiles * h.batch;
     p.total_tiles = int(tiles);
+    p.group_m = CTAS == 2 ? 8 : 16;  // about sqrt(concurrent tiles) rows per group
     const int64_t units_max = sm_count() / CTAS;
     const int units = int(tiles < units_max ? tiles : units_max);
     return launch_pdl(kern, units * CTAS, kThreads, L::kAlloc, st, CTAS, ta, tb, tc, p);
