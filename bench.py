@@ -45,6 +45,33 @@ E4M3, E5M2 = 0, 1
 NT, NN, TN = 0, 1, 2
 
 
+KERNEL_SOURCES = {
+    "gemm": ("gemm.cu", "sm100.cuh", "common.cuh"),
+    "quantize": ("quantize.cu", "common.cuh"),
+}
+
+
+def source_hash(kind):
+    """sha256 over the CUDA sources a kernel family is built from."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kind]:
+        with open(os.path.join(ROOT, "fp8_delayed_scaling_quantize_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(kind):
+    """DRAM bytes per launch from the committed ncu capture summary, or None
+    when the kernel's sources changed since the capture."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)[kind]
+    except Exception:
+        return None
+    return t["dram_bytes_per_launch"] if t.get("source_sha256") == source_hash(kind) else None
+
+
 def _peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -354,14 +381,14 @@ def run_ours(args, world, rank, local):
         "quantize_gbs": round(quant_gbs, 1),
         "roofline": {"bound": "tensor", "achieved": round(gemm_tf, 1), "peak": round(fp8_burst, 1),
                      "unit": "TFLOP/s", "frac": round(gemm_tf / fp8_burst, 4),
-                     "traffic": None,
+                     "traffic": measured_traffic("gemm"),
                      "kernel": "fp8_gemm_kernel (all 12 GEMM launches of a step, FLOP-weighted)",
                      "peak_source": f"{peak_src}: 2 x bf16 burst {bf16_burst} TF/s (nominal fp8:bf16 = 2)",
                      "algorithmic_bytes_per_launch": round(g_bytes / n_g),
                      "flops_per_launch": round(g_flops / n_g),
                      "avg_launch_us": round(1e3 * g_ms / n_g, 2)},
         "roofline_quantize": {"bound": "hbm", "achieved": round(quant_gbs, 1), "peak": hbm, "unit": "GB/s",
-                              "frac": round(quant_gbs / hbm, 4), "traffic": None,
+                              "frac": round(quant_gbs / hbm, 4), "traffic": measured_traffic("quantize"),
                               "kernel": "quantize_kernel (delayed, 12 launches per step)",
                               "peak_source": f"{peak_src} hbm copy",
                               "algorithmic_bytes_per_launch": round(3 * q_elems / n_q),
