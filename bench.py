@@ -363,6 +363,7 @@ def run_ours(args, world, rank, local):
         e2e = run_e2e(fp8, stack, stream, args.e2e_steps, world, side)
         e2e["value"] = round(e2e["value"], 3)
 
+    context = {} if args.no_compare else compare_bf16(stack, ms_step, 200)
     gpu_launches = 24 * args.steps
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
@@ -395,6 +396,7 @@ def run_ours(args, world, rank, local):
                               "avg_launch_us": round(1e3 * q_ms / n_q, 2)},
         "gemm_by_shape": gemm_detail,
         "clocks": clocks.summary(),
+        "context": context,
         "e2e": e2e,
         "gpu_launches": gpu_launches,
     }
@@ -402,6 +404,91 @@ def run_ours(args, world, rank, local):
         line["cpu_baseline"] = cpu_baseline_full_step()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def _graph_time(fn, stream, reps, warm=3):
+    """Capture fn() in a CUDA graph on `stream`; return ms per replay."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for _ in range(warm):
+            fn()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for _ in range(warm):
+            g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+    e1.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    del g
+    return ms
+
+
+def compare_bf16(stack, fp8_ms, reps):
+    """The same linear-stack training step as bf16 GEMMs on cuBLAS
+    (torch.matmul; forward, then dX and dW in reverse, dW on a second
+    stream), and the step through the autograd layer (Fp8Linear vs bf16
+    nn.Linear), each as a CUDA graph: the FP8-over-bf16 speed-up the
+    AstrAI commit logs report for their kernels."""
+    out = {}
+    T = W.TOKENS
+    ts = stack.sets[0]
+    ys = [torch.empty(T, L["d_out"], dtype=torch.bfloat16, device="cuda") for L in stack.lin]
+    dxs = [torch.empty(T, L["d_in"], dtype=torch.bfloat16, device="cuda") for L in stack.lin]
+    dws = [torch.empty(L["d_out"], L["d_in"], dtype=torch.bfloat16, device="cuda") for L in stack.lin]
+    side = torch.cuda.Stream()
+
+    def bf16_step():
+        cur = torch.cuda.current_stream()
+        for li, t in enumerate(ts):
+            torch.matmul(t["x"], t["w"].t(), out=ys[li])
+        for li in reversed(range(len(ts))):
+            t = ts[li]
+            side.wait_stream(cur)
+            with torch.cuda.stream(side):
+                torch.matmul(t["g"].t(), t["x"], out=dws[li])
+            torch.matmul(t["g"], t["w"], out=dxs[li])
+            cur.wait_stream(side)
+
+    st = torch.cuda.Stream()
+    bf16_ms = _graph_time(bf16_step, st, reps)
+    out["bf16_cublas_step_ms"] = round(bf16_ms, 4)
+    out["fp8_over_bf16_step"] = round(bf16_ms / fp8_ms, 3)
+
+    # through torch.autograd: Fp8Linear vs bf16 nn.Linear, forward + backward
+    try:
+        from fp8_delayed_scaling_quantize_b200.linear import Fp8Linear
+        mods8 = [Fp8Linear(L["d_in"], L["d_out"], bias=False, device="cuda") for L in stack.lin]
+        mods16 = [torch.nn.Linear(L["d_in"], L["d_out"], bias=False, device="cuda", dtype=torch.bfloat16)
+                  for L in stack.lin]
+        xs = [t["x"].detach().clone().requires_grad_(True) for t in ts]
+        gs = [t["g"] for t in ts]
+
+        def ag_step(mods):
+            def fn():
+                for m in mods:
+                    m.weight.grad = None
+                for x in xs:
+                    x.grad = None
+                ys_ = [m(x) for m, x in zip(mods, xs)]
+                torch.autograd.backward(ys_, gs)
+            return fn
+
+        out["autograd_fp8_step_ms"] = round(_graph_time(ag_step(mods8), st, reps), 4)
+        out["autograd_bf16_step_ms"] = round(_graph_time(ag_step(mods16), st, reps), 4)
+        out["autograd_fp8_over_bf16"] = round(out["autograd_bf16_step_ms"] / out["autograd_fp8_step_ms"], 3)
+    except Exception as e:  # capture failures are reported, not hidden
+        out["autograd_error"] = f"{type(e).__name__}: {e}"[:200]
+    return out
 
 
 def run_e2e(fp8, stack, stream, steps, world, side=None):
@@ -623,6 +710,7 @@ def main():
     ap.add_argument("--one-stream", action="store_true", help="issue the whole step on one stream")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-compare", action="store_true", help="skip the bf16 / autograd comparison")
     ap.add_argument("--breakdown-reps", type=int, default=20)
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--kernel", choices=["gemm", "quantize", "cublaslt"], help="single-kernel mode")

@@ -57,6 +57,7 @@ def _load():
         "fp8_mm": (I, [P, I, P, I, P, P, I, I64, I64, I64, I64, I64, I64, I64, P, P, I, P, P]),
         "fp8_last_device_error": (I, []),
         "fp8_selftest_wait_timeout": (I, [ctypes.c_uint32, P]),
+        "fp8_bias_grad": (I, [P, I64, I64, P, P]),
     }
     for name, (res, args) in sig.items():
         try:
@@ -132,6 +133,10 @@ def fp8_mm(a8, fa, b8, fb, sa, sb, layout, M, N, K, batch, stride_a, stride_b, s
 
 def fp8_last_device_error():
     return _check(lib.fp8_last_device_error(), "fp8_last_device_error")
+
+
+def fp8_bias_grad(g, rows, cols, out, stream=None):
+    return _check(lib.fp8_bias_grad(_ptr(g), int(rows), int(cols), _ptr(out), _stream(stream)), "fp8_bias_grad")
 
 
 def fp8_selftest_wait_timeout(limit_us: int, stream=None):

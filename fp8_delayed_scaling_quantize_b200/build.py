@@ -14,7 +14,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libfp8lite.so")
-SOURCES = ("quantize.cu", "gemm.cu")
+SOURCES = ("quantize.cu", "gemm.cu", "colsum.cu")
 
 
 NVCC_FLAGS = [

@@ -175,6 +175,18 @@ FP8LITE_API fp8_status fp8_mm(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8, 
  * FP8_OK otherwise, FP8_ERR_CUDA if the synchronisation failed. */
 FP8LITE_API fp8_status fp8_last_device_error(void);
 
+/* Bias gradient of a linear layer: out[j] = bf16_rne( sum_i g[i][j] ), the
+ * sum over the rows (tokens, leading dimensions flattened) accumulated in
+ * fp32 [fp8.py@f4c44ebf, bullets on the bias column-sum and the 3-D
+ * backward]. It is a separate call so that it runs only when the bias needs
+ * a gradient, and it reads the bf16 gradient (not its FP8 codes).
+ * g    device bf16[rows * cols], row-major, 4-byte aligned
+ * out  device bf16[cols], 2-byte aligned
+ * rows >= 1, cols >= 1 and even.
+ * Errors: FP8_ERR_INVALID_ARG, FP8_ERR_ALIGNMENT (odd cols, misaligned
+ *         pointers), FP8_ERR_CUDA. */
+FP8LITE_API fp8_status fp8_bias_grad(const void* g, int64_t rows, int64_t cols, void* out, void* stream);
+
 /* Diagnostic of the failure path: launches one tiny kernel whose single
  * thread waits, through the same bounded wait the GEMM uses, on a barrier
  * that nothing arrives at. After limit_us (1 .. 1e6 microseconds) the wait

@@ -62,3 +62,8 @@ from .gemm import (  # noqa: F401
     mm_sampled,
     tolerance,
 )
+from .linear import (  # noqa: F401
+    bias_grad,
+    bias_grad_tolerance,
+    Fp8LinearRef,
+)
