@@ -5,10 +5,12 @@ stack at 2048 tokens (B4 x T512): for each of the 4 linears (QKV 1024->3072,
 out 1024->1024, MLP 1024->4096, 4096->1024) delayed-scaling quantize of x
 and W to E4M3 and of the gradient g to E5M2 (ring finalized in-kernel),
 then the forward NT GEMM y = x W^T, the dX NN GEMM g W and the dW TN GEMM
-g^T x -- 12 quantize launches and 12 GEMM launches, all through the C ABI.
+g^T x, all through the C ABI: 12 GEMM launches and 8 quantize launches (one
+grouped launch for every W and the first x, then each later x and every g;
+--no-grouped: 12 single-tensor quantize launches).
 
 value  = GEMM FLOPs of the step (154.6 GFLOP) / device step time, TFLOP/s,
-         the step replayed as one CUDA graph (24 kernel nodes), inputs
+         the step replayed as one CUDA graph (20 kernel nodes), inputs
          resident in HBM, rotating through 3 input sets (276 MB > 126 MB L2).
 e2e    = the same metric through the public API with HOST buffers: pinned
          host -> device copies of x, W, g and device -> host copies of y,
@@ -171,7 +173,7 @@ class ClockSampler:
 # ------------------------------------------------------------- the stack ---
 
 class Stack:
-    """Device buffers and the 24 C-ABI calls of one step of the linear stack."""
+    """Device buffers and the C-ABI calls of one step of the linear stack."""
 
     def __init__(self, fp8, n_sets=N_SETS, dev="cuda"):
         self.fp8 = fp8
@@ -220,21 +222,34 @@ class Stack:
         L = self.lin[li]
         return 2 * W.TOKENS * L["d_in"] * L["d_out"]
 
-    def step(self, s, stream, side=None):
+    def grouped_call(self, s):
+        """The step-start quantize of every linear's W and of the first x,
+        as the jobs of one fp8_quantize_many launch."""
+        return [self.quant_calls(s, li)[1] for li in range(len(self.lin))] + [self.quant_calls(s, 0)[0]]
+
+    def step(self, s, stream, side=None, grouped=True):
         """Issue one training step of the stack on input set s: the forward
         of every linear in order (quantize x and W, y = x W^T), then the
         backward in reverse order (quantize g, dX = g W, dW = g^T x).
 
+        grouped: the weights are all known when the step starts, so every W
+        and the first x are quantized by one grouped launch; the x of later
+        linears and every g still wait for the layer before them.
         With a `side` stream, the work a linear layer can overlap runs on it:
-        W's quantize beside x's, and dW beside dX (both only need g8); the
-        streams fork and join around each pair, so the dependencies between
-        linears are those of a sequential model."""
+        W's quantize beside x's (ungrouped), and dW beside dX (both only need
+        g8); the streams fork and join around each pair, so the dependencies
+        between linears are those of a sequential model."""
         fp8 = self.fp8
         n = len(self.lin)
+        if grouped:
+            fp8.fp8_quantize_many(self.grouped_call(s), stream=stream)
         for li in range(n):
             qx, qw, _ = self.quant_calls(s, li)
             fwd, _, _ = self.gemm_calls(li)
-            if side is not None:
+            if grouped:
+                if li > 0:
+                    fp8.fp8_quantize(*qx, stream=stream)
+            elif side is not None:
                 side.wait_stream(stream)
                 fp8.fp8_quantize(*qw, stream=side)
                 fp8.fp8_quantize(*qx, stream=stream)
@@ -255,6 +270,10 @@ class Stack:
             else:
                 fp8.fp8_mm(*dx, stream=stream)
                 fp8.fp8_mm(*dw, stream=stream)
+
+    def launches_per_step(self, grouped=True):
+        n = len(self.lin)
+        return 3 * n + (1 + (n - 1) + n if grouped else 3 * n)
 
 
 def hold_stream(stream, us=2000):
@@ -279,12 +298,13 @@ def run_ours(args, world, rank, local):
     stream = torch.cuda.Stream()
     side = None if args.one_stream else torch.cuda.Stream()
     stack = Stack(fp8)
+    grouped = not args.no_grouped
     torch.cuda.synchronize()
 
     # warm-up (eager) also sets kernel attributes before any capture
     with torch.cuda.stream(stream):
         for i in range(max(args.warmup, 3)):
-            stack.step(i % N_SETS, stream, side)
+            stack.step(i % N_SETS, stream, side, grouped)
     torch.cuda.synchronize()
 
     graphs = []
@@ -292,7 +312,7 @@ def run_ours(args, world, rank, local):
         for s in range(N_SETS):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
-                stack.step(s, stream, side)
+                stack.step(s, stream, side, grouped)
             graphs.append(g)
         torch.cuda.synchronize()
         for i in range(max(args.warmup, 3)):
@@ -321,7 +341,7 @@ def run_ours(args, world, rank, local):
     value = weak_scaling_value(stack.flops, args.steps, world, t_ms)
 
     # ---- per-kernel breakdown -----------------------------------------
-    # Each of the step's 24 launches is repeated back to back between one
+    # Each of the step's 12 quantizes and 12 GEMMs is repeated back to back between one
     # event pair (the stream held while the host enqueues), so the average is
     # the kernel's steady-state cost on the stream, as inside the graph.
     q_ms = g_ms = 0.0
@@ -352,6 +372,30 @@ def run_ours(args, world, rank, local):
                 g_bytes += gemm_algorithmic_bytes(c[6], M, N, K)
                 n_g += 1
                 per_shape[f"{'NT NN TN'.split()[c[6]]} {M}x{N}x{K}"] = (ms, 2 * M * N * K)
+    # the grouped step-start launch (all W + the first x) against its
+    # tensors quantized one launch each
+    jobs = stack.grouped_call(0)
+    hold_stream(stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        fp8.fp8_quantize_many(jobs, stream=stream)
+    e1.record(stream)
+    e1.synchronize()
+    many_ms = e0.elapsed_time(e1) / reps
+    many_elems = sum(j[1] for j in jobs)
+    hold_stream(stream)
+    e0.record(stream)
+    for _ in range(reps):
+        for j in jobs:
+            fp8.fp8_quantize(*j, stream=stream)
+    e1.record(stream)
+    e1.synchronize()
+    single_ms = e0.elapsed_time(e1) / reps
+    grouped_detail = {"jobs": len(jobs), "elems": many_elems, "us": round(1e3 * many_ms, 2),
+                      "gbs": round(3.0 * many_elems / (many_ms * 1e-3) / 1e9, 1),
+                      "frac": round(3.0 * many_elems / (many_ms * 1e-3) / 1e9 / hbm, 4),
+                      "same_tensors_one_launch_each_us": round(1e3 * single_ms, 2)}
     gemm_tf = g_flops / (g_ms * 1e-3) / 1e12
     quant_gbs = 3.0 * q_elems / (q_ms * 1e-3) / 1e9
     gemm_detail = {k: {"us": round(1e3 * ms, 2), "tflops": round(f / (ms * 1e-3) / 1e12, 1)}
@@ -360,11 +404,11 @@ def run_ours(args, world, rank, local):
     # ---- e2e: host buffers through the public API ------------------------
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(fp8, stack, stream, args.e2e_steps, world, side)
+        e2e = run_e2e(fp8, stack, stream, args.e2e_steps, world, side, grouped)
         e2e["value"] = round(e2e["value"], 3)
 
     context = {} if args.no_compare else compare_bf16(stack, ms_step, 200)
-    gpu_launches = 24 * args.steps
+    gpu_launches = stack.launches_per_step(grouped) * args.steps
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
@@ -376,7 +420,10 @@ def run_ours(args, world, rank, local):
                    "quant_elems_per_step": stack.q_elems,
                    "l2": f"{N_SETS} rotating input sets ({N_SETS * 2 * stack.q_elems / 1e6:.0f} MB bf16) > 126 MB L2",
                    "launch": ("CUDA graph per step" if graphs else "eager") +
-                             (", 1 stream" if side is None else ", 2 streams (x||W quantize, dX||dW)"),
+                             (", 1 stream" if side is None else
+                              ", 2 streams (dX||dW" + (")" if grouped else ", x||W quantize)")) +
+                             (", all W + first x quantized in one grouped launch" if grouped else ""),
+                   "launches_per_step": stack.launches_per_step(grouped),
                    "order": "forward over linears, then backward in reverse",
                    "parallelism": f"replicas x{world}"},
         "quantize_gbs": round(quant_gbs, 1),
@@ -395,6 +442,7 @@ def run_ours(args, world, rank, local):
                               "algorithmic_bytes_per_launch": round(3 * q_elems / n_q),
                               "avg_launch_us": round(1e3 * q_ms / n_q, 2)},
         "gemm_by_shape": gemm_detail,
+        "quantize_grouped": grouped_detail,
         "clocks": clocks.summary(),
         "context": context,
         "e2e": e2e,
@@ -491,8 +539,8 @@ def compare_bf16(stack, fp8_ms, reps):
     return out
 
 
-def run_e2e(fp8, stack, stream, steps, world, side=None):
-    """H2D of the step's inputs from pinned host memory, the 24 calls, D2H of
+def run_e2e(fp8, stack, stream, steps, world, side=None, grouped=True):
+    """H2D of the step's inputs from pinned host memory, the step's calls, D2H of
     the three GEMM outputs, per step; CUDA events around the whole loop."""
     host_in = [{k: v.cpu().pin_memory() for k, v in t.items()} for t in stack.sets[0]]
     host_out = [{k: torch.empty(L[k].numel(), dtype=torch.bfloat16).pin_memory() for k in ("y", "dx", "dw")}
@@ -504,7 +552,7 @@ def run_e2e(fp8, stack, stream, steps, world, side=None):
         for li, t in enumerate(host_in):
             for k, v in t.items():
                 stack.sets[0][li][k].copy_(v, non_blocking=True)
-        stack.step(0, stream, side)
+        stack.step(0, stream, side, grouped)
         for li, L in enumerate(stack.lin):
             for k in ("y", "dx", "dw"):
                 host_out[li][k].copy_(L[k], non_blocking=True)
@@ -708,6 +756,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--one-stream", action="store_true", help="issue the whole step on one stream")
+    ap.add_argument("--no-grouped", action="store_true", help="quantize every tensor with its own launch")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-compare", action="store_true", help="skip the bf16 / autograd comparison")

@@ -41,6 +41,15 @@ class fp8_ring(ctypes.Structure):
 
 assert ctypes.sizeof(fp8_ring) == FP8_RING_BYTES
 
+FP8_QUANTIZE_MAX_JOBS = 8
+
+
+class fp8_quantize_job(ctypes.Structure):
+    """One job of fp8_quantize_many (pointers are device addresses)."""
+    _fields_ = [("x", ctypes.c_void_p), ("n", ctypes.c_int64), ("fmt", ctypes.c_int32),
+                ("ring", ctypes.c_void_p), ("out8", ctypes.c_void_p), ("amax_out", ctypes.c_void_p),
+                ("scale_out", ctypes.c_void_p)]
+
 
 def _load():
     if not os.path.exists(LIB_PATH):
@@ -58,6 +67,7 @@ def _load():
         "fp8_last_device_error": (I, []),
         "fp8_selftest_wait_timeout": (I, [ctypes.c_uint32, P]),
         "fp8_bias_grad": (I, [P, I64, I64, P, P]),
+        "fp8_quantize_many": (I, [P, ctypes.c_int32, P]),
     }
     for name, (res, args) in sig.items():
         try:
@@ -121,6 +131,16 @@ def fp8_ring_set(ring, host: fp8_ring, stream=None):
 def fp8_quantize(x, n, fmt, ring, out8, amax_out, scale_out, stream=None):
     return _check(lib.fp8_quantize(_ptr(x), int(n), int(fmt), _ptr(ring), _ptr(out8), _ptr(amax_out),
                                    _ptr(scale_out), _stream(stream)), "fp8_quantize")
+
+
+def fp8_quantize_many(jobs, stream=None):
+    """jobs: sequence of (x, n, fmt, ring, out8, amax_out, scale_out)."""
+    arr = (fp8_quantize_job * max(len(jobs), 1))()
+    for i, (x, n, fmt, ring, out8, amax_out, scale_out) in enumerate(jobs):
+        arr[i] = fp8_quantize_job(_ptr(x), int(n), int(fmt), _ptr(ring), _ptr(out8), _ptr(amax_out),
+                                  _ptr(scale_out))
+    return _check(lib.fp8_quantize_many(ctypes.cast(arr, ctypes.c_void_p), len(jobs), _stream(stream)),
+                  "fp8_quantize_many")
 
 
 def fp8_mm(a8, fa, b8, fb, sa, sb, layout, M, N, K, batch, stride_a, stride_b, stride_c, bias,

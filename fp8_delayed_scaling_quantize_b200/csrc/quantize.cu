@@ -96,16 +96,17 @@ __device__ __forceinline__ uint32_t block_max_bits(float m) {
     return bits;
 }
 
+// The quantize pass of one tensor, run by block `blk` of the `nblk` blocks
+// given to it (a whole grid for fp8_quantize, a share of one for
+// fp8_quantize_many). s_scale is the block's shared scale slot.
 template <int FMT, int MODE>
-__global__ void __launch_bounds__(kThreads)
-quantize_kernel(const uint16_t* __restrict__ x, int64_t n, uint8_t* __restrict__ out8,
-                fp8_ring* ring, uint32_t* amax_acc, float* amax_out, float* scale_out) {
+__device__ __forceinline__ void quantize_body(const uint16_t* __restrict__ x, int64_t n, uint8_t* __restrict__ out8,
+                                              fp8_ring* ring, uint32_t* amax_acc, float* amax_out, float* scale_out,
+                                              int blk, int nblk, float& s_scale) {
     const float fmax = fmt_max(FMT);
-    griddep_wait();  // inputs and the ring come from earlier kernels
     // One thread per block reads the scale (or the amax it comes from) and
     // shares it: thousands of warps loading one address would queue on a
     // single L2 line.
-    __shared__ float s_scale;
     if (MODE != kAmaxOnly) {
         if (threadIdx.x == 0) {
             float v;
@@ -116,7 +117,7 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t n, uint8_t* __restrict__
                 v = (a > 0.0f && isfinite(a)) ? scale_from_amax(fmax, a) : 1.0f;
             }
             s_scale = v;
-            if (blockIdx.x == 0) *scale_out = v;
+            if (blk == 0) *scale_out = v;
         }
         __syncthreads();
     }
@@ -125,8 +126,8 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t n, uint8_t* __restrict__
     const uint4* xv = reinterpret_cast<const uint4*>(x);
     uint2* ov = reinterpret_cast<uint2*>(out8);
     const int64_t units = n >> 3;  // 8 elements per unit
-    const int64_t tid = int64_t(blockIdx.x) * kThreads + threadIdx.x;
-    const int64_t stride = int64_t(gridDim.x) * kThreads;
+    const int64_t tid = int64_t(blk) * kThreads + threadIdx.x;
+    const int64_t stride = int64_t(nblk) * kThreads;
     float m = 0.0f;
 
     for (int64_t base = tid; base < units; base += stride * kUnroll) {
@@ -172,7 +173,7 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t n, uint8_t* __restrict__
     // ticket with acquire-release semantics (its amax is visible before the
     // ticket moves); the block holding the final ticket sees every amax.
     const uint32_t ticket = atom_add_acq_rel(&ring->ticket, 1u);
-    if (ticket != gridDim.x - 1) return;
+    if (ticket != uint32_t(nblk) - 1) return;
     const float a = __uint_as_float(atomicExch(&ring->amax_bits, 0u));
     volatile fp8_ring* r = ring;
     // the window's maximum over the 15 kept entries and the new amax; the
@@ -190,6 +191,45 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t n, uint8_t* __restrict__
     r->idx = (idx + 1) & (FP8_RING_HISTORY - 1);
     if (amax_out) *amax_out = a;
     r->ticket = 0u;  // ready for the next call (visible at the kernel boundary)
+}
+
+template <int FMT, int MODE>
+__global__ void __launch_bounds__(kThreads)
+quantize_kernel(const uint16_t* __restrict__ x, int64_t n, uint8_t* __restrict__ out8,
+                fp8_ring* ring, uint32_t* amax_acc, float* amax_out, float* scale_out) {
+    __shared__ float s_scale;
+    griddep_wait();  // inputs and the ring come from earlier kernels
+    quantize_body<FMT, MODE>(x, n, out8, ring, amax_acc, amax_out, scale_out, blockIdx.x, gridDim.x, s_scale);
+}
+
+// Several delayed-scaling quantizations in one launch: job j owns blocks
+// [first[j], first[j] + blocks[j]) of the grid and runs exactly what
+// fp8_quantize does for it, its ring finalized by the last of its blocks.
+struct QuantJobs {
+    int count;
+    int first[FP8_QUANTIZE_MAX_JOBS];
+    int blocks[FP8_QUANTIZE_MAX_JOBS];
+    int fmt[FP8_QUANTIZE_MAX_JOBS];
+    const uint16_t* x[FP8_QUANTIZE_MAX_JOBS];
+    int64_t n[FP8_QUANTIZE_MAX_JOBS];
+    fp8_ring* ring[FP8_QUANTIZE_MAX_JOBS];
+    uint8_t* out8[FP8_QUANTIZE_MAX_JOBS];
+    float* amax_out[FP8_QUANTIZE_MAX_JOBS];
+    float* scale_out[FP8_QUANTIZE_MAX_JOBS];
+};
+
+__global__ void __launch_bounds__(kThreads) quantize_many_kernel(const __grid_constant__ QuantJobs jobs) {
+    __shared__ float s_scale;
+    griddep_wait();
+    int j = 0;
+    while (j + 1 < jobs.count && int(blockIdx.x) >= jobs.first[j + 1]) ++j;
+    const int blk = int(blockIdx.x) - jobs.first[j];
+    if (jobs.fmt[j] == FP8_E4M3)
+        quantize_body<FP8_E4M3, kDelayed>(jobs.x[j], jobs.n[j], jobs.out8[j], jobs.ring[j], nullptr,
+                                          jobs.amax_out[j], jobs.scale_out[j], blk, jobs.blocks[j], s_scale);
+    else
+        quantize_body<FP8_E5M2, kDelayed>(jobs.x[j], jobs.n[j], jobs.out8[j], jobs.ring[j], nullptr,
+                                          jobs.amax_out[j], jobs.scale_out[j], blk, jobs.blocks[j], s_scale);
 }
 
 __global__ void ring_write_kernel(fp8_ring* ring, fp8_ring value) {
@@ -302,4 +342,33 @@ extern "C" fp8_status fp8_quantize(const void* x, int64_t n, fp8_fmt fmt, fp8_ri
     cudaStream_t st = as_stream(stream);
     return fmt == FP8_E4M3 ? launch_quantize<FP8_E4M3>(xb, n, ring, out8, amax_out, scale_out, st)
                            : launch_quantize<FP8_E5M2>(xb, n, ring, out8, amax_out, scale_out, st);
+}
+
+extern "C" fp8_status fp8_quantize_many(const fp8_quantize_job* jobs, int32_t count, void* stream) {
+    if (!jobs || count < 1 || count > FP8_QUANTIZE_MAX_JOBS) return FP8_ERR_INVALID_ARG;
+    QuantJobs q = {};
+    q.count = count;
+    int total = 0;
+    for (int j = 0; j < count; ++j) {
+        const fp8_quantize_job& in = jobs[j];
+        if (!valid_fmt(in.fmt)) return FP8_ERR_INVALID_ARG;
+        if (in.n < 0 || in.n >= (int64_t(1) << 40)) return FP8_ERR_INVALID_ARG;
+        if (!in.ring || !in.scale_out) return FP8_ERR_INVALID_ARG;
+        if (in.n > 0 && (!in.x || !in.out8)) return FP8_ERR_INVALID_ARG;
+        if (!aligned(in.x, 16) || !aligned(in.out8, 16)) return FP8_ERR_ALIGNMENT;
+        if (!aligned(in.ring, 4) || !aligned(in.scale_out, 4) || !aligned(in.amax_out, 4)) return FP8_ERR_ALIGNMENT;
+        for (int k = 0; k < j; ++k)
+            if (jobs[k].ring == in.ring) return FP8_ERR_INVALID_ARG;  // one ring, one call at a time
+        q.first[j] = total;
+        q.blocks[j] = grid_for(in.n);
+        total += q.blocks[j];
+        q.fmt[j] = int(in.fmt);
+        q.x[j] = static_cast<const uint16_t*>(in.x);
+        q.n[j] = in.n;
+        q.ring[j] = in.ring;
+        q.out8[j] = in.out8;
+        q.amax_out[j] = in.amax_out;
+        q.scale_out[j] = in.scale_out;
+    }
+    return launch_pdl(quantize_many_kernel, total, kThreads, 0, as_stream(stream), 1, q);
 }

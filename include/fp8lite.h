@@ -131,6 +131,26 @@ FP8LITE_API fp8_status fp8_quantize(const void* x, int64_t n, fp8_fmt fmt, fp8_r
                         uint8_t* out8, float* amax_out, float* scale_out,
                         void* stream);
 
+/* Several delayed-scaling quantizations in ONE launch, e.g. the weights of
+ * all layers at the start of a training step, or a layer's x and W.
+ * Each job is exactly an fp8_quantize call with a ring (same arguments, same
+ * results, its ring finalized by the last of the job's thread blocks); the
+ * jobs run concurrently. Jobs must use distinct rings and must not overlap
+ * in their outputs; current scaling (no ring) is not offered here.
+ * count: 1 .. FP8_QUANTIZE_MAX_JOBS. Errors as fp8_quantize, plus
+ * FP8_ERR_INVALID_ARG for a bad count, a NULL ring or a ring used twice. */
+#define FP8_QUANTIZE_MAX_JOBS 8
+typedef struct fp8_quantize_job {
+    const void* x;     /* device bf16[n], 16-byte aligned */
+    int64_t n;         /* 0 <= n < 2^40 */
+    int32_t fmt;       /* fp8_fmt */
+    fp8_ring* ring;    /* required */
+    uint8_t* out8;     /* device uint8[n], 16-byte aligned */
+    float* amax_out;   /* optional */
+    float* scale_out;  /* required: the scale this job used */
+} fp8_quantize_job;
+FP8LITE_API fp8_status fp8_quantize_many(const fp8_quantize_job* jobs, int32_t count, void* stream);
+
 /* Per-tensor-scaled FP8 GEMM with fused bias and bf16 output
  * [fp8.py@f4c44ebf, bullets on the fused bias and 3-D operands;
  *  mma@cebdd45d, bullet on the bias_scale slot].

@@ -108,3 +108,18 @@ def test_ring_validation(fp8):
     host.scale = 1.0
     assert fp8.raw_status("fp8_ring_set", S, ctypes.byref(host), None) == fp8.FP8_ERR_INVALID_ARG
     assert fp8.raw_status("fp8_ring_get", None, ctypes.byref(host), None) == fp8.FP8_ERR_INVALID_ARG
+
+
+def test_quantize_many_validation(fp8):
+    def status(jobs, count=None):
+        arr = (fp8.fp8_quantize_job * max(len(jobs), 1))(*[fp8.fp8_quantize_job(*j) for j in jobs])
+        return fp8.raw_status("fp8_quantize_many", ctypes.cast(arr, ctypes.c_void_p),
+                              len(jobs) if count is None else count, None)
+    good = (A, 64, 0, S, A + 4096, None, S + 64)
+    assert status([good], count=0) == fp8.FP8_ERR_INVALID_ARG
+    assert status([good] * 9) == fp8.FP8_ERR_INVALID_ARG
+    assert status([good, good]) == fp8.FP8_ERR_INVALID_ARG                    # one ring twice
+    assert status([(A, 64, 0, None, A + 4096, None, S + 64)]) == fp8.FP8_ERR_INVALID_ARG  # no ring
+    assert status([(A, 64, 5, S, A + 4096, None, S + 64)]) == fp8.FP8_ERR_INVALID_ARG     # bad fmt
+    assert status([(A + 2, 64, 0, S, A + 4096, None, S + 64)]) == fp8.FP8_ERR_ALIGNMENT
+    assert fp8.raw_status("fp8_quantize_many", None, 1, None) == fp8.FP8_ERR_INVALID_ARG

@@ -189,3 +189,29 @@ def test_misaligned_input_is_rejected(g):
     st = fp8.raw_status("fp8_quantize", x.data_ptr() + 2, 32, 0, None, out.data_ptr(),
                         amax.data_ptr(), amax.data_ptr(), None)
     assert st == fp8.FP8_ERR_ALIGNMENT
+
+
+def test_quantize_many_matches_the_oracle_per_job(g):
+    """One launch quantizing several tensors (mixed formats, ragged, empty)
+    equals fp8_quantize on each, over repeated calls (rings evolve)."""
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    sizes = [(3 << 20) + 5, 1000, 0, (1 << 18) + 3, 4096 * 37]
+    fmts = [E4M3, E5M2, E4M3, E5M2, E4M3]
+    rings = [g.new_ring() for _ in sizes]
+    refs = [oracle.DelayedRing() for _ in sizes]
+    outs = [torch.empty(max(n, 1), dtype=torch.uint8, device="cuda") for n in sizes]
+    amaxs = [torch.empty(1, device="cuda") for _ in sizes]
+    scales = [torch.empty(1, device="cuda") for _ in sizes]
+    for call in range(3):
+        xs = [(W.bf16_normal((n,), 0.5, 8000 + 10 * call + j).float() * (j + 1) * (call + 1)).to(torch.bfloat16)
+              for j, n in enumerate(sizes)]
+        xd = [x.cuda() for x in xs]
+        fp8.fp8_quantize_many([(xd[j] if sizes[j] else None, sizes[j], fmts[j], rings[j],
+                                outs[j] if sizes[j] else None, amaxs[j], scales[j]) for j in range(len(sizes))])
+        for j, n in enumerate(sizes):
+            want, a, s = refs[j].step(xs[j].float().numpy(), fmts[j])
+            assert np.array_equal(g.codes(outs[j])[:n], want), (call, j)
+            assert g.f32(scales[j])[0] == s and g.f32(amaxs[j])[0] == a, (call, j)
+            hist, rs, idx, acc, ticket = g.ring_state(rings[j])
+            assert np.array_equal(hist, refs[j].hist) and rs == refs[j].scale and idx == refs[j].idx
+            assert acc == 0 and ticket == 0
