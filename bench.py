@@ -199,6 +199,24 @@ class Stack:
             self.lin.append(L)
         self.flops = W.stack_flops()
         self.q_elems = W.stack_quant_elems()
+        self.split_k = 0
+        self.ws = [None, None]
+
+    def use_split(self, split_k):
+        """Run every GEMM of the step that can take it with split_k K-splits,
+        one zero-filled workspace per stream."""
+        self.split_k = split_k
+        if split_k > 1:
+            need = max(self.fp8.fp8_mm_workspace_size(*c[7:11], c[6], split_k) for li in range(len(self.lin))
+                       for c in self.gemm_calls(li))
+            self.ws = [torch.zeros(max(need, 4096), dtype=torch.uint8, device=self.dev) for _ in range(2)]
+
+    def mm(self, call, stream, ws_index=0):
+        c = call
+        if self.split_k > 1 and self.fp8.fp8_mm_workspace_size(*c[7:11], c[6], self.split_k) > 0:
+            self.fp8.fp8_mm_ws(*call, self.ws[ws_index], self.split_k, stream=stream)
+        else:
+            self.fp8.fp8_mm(*call, stream=stream)
 
     def quant_calls(self, s, li):
         L, t = self.lin[li], self.sets[s][li]
@@ -257,19 +275,19 @@ class Stack:
             else:
                 fp8.fp8_quantize(*qx, stream=stream)
                 fp8.fp8_quantize(*qw, stream=stream)
-            fp8.fp8_mm(*fwd, stream=stream)
+            self.mm(fwd, stream)
         for li in reversed(range(n)):
             _, _, qg = self.quant_calls(s, li)
             _, dx, dw = self.gemm_calls(li)
             fp8.fp8_quantize(*qg, stream=stream)
             if side is not None:
                 side.wait_stream(stream)
-                fp8.fp8_mm(*dw, stream=side)
-                fp8.fp8_mm(*dx, stream=stream)
+                self.mm(dw, side, 1)
+                self.mm(dx, stream, 0)
                 stream.wait_stream(side)
             else:
-                fp8.fp8_mm(*dx, stream=stream)
-                fp8.fp8_mm(*dw, stream=stream)
+                self.mm(dx, stream)
+                self.mm(dw, stream)
 
     def launches_per_step(self, grouped=True):
         n = len(self.lin)
@@ -298,6 +316,7 @@ def run_ours(args, world, rank, local):
     stream = torch.cuda.Stream()
     side = None if args.one_stream else torch.cuda.Stream()
     stack = Stack(fp8)
+    stack.use_split(args.split_k)
     grouped = not args.no_grouped
     torch.cuda.synchronize()
 
@@ -352,12 +371,14 @@ def run_ours(args, world, rank, local):
     for li in range(len(stack.lin)):
         calls = [("quantize", c) for c in stack.quant_calls(0, li)] + [("gemm", c) for c in stack.gemm_calls(li)]
         for kind, c in calls:
-            fn = fp8.fp8_quantize if kind == "quantize" else fp8.fp8_mm
             hold_stream(stream)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             for _ in range(reps):
-                fn(*c, stream=stream)
+                if kind == "quantize":
+                    fp8.fp8_quantize(*c, stream=stream)
+                else:
+                    stack.mm(c, stream)
             e1.record(stream)
             e1.synchronize()
             ms = e0.elapsed_time(e1) / reps
@@ -422,7 +443,8 @@ def run_ours(args, world, rank, local):
                    "launch": ("CUDA graph per step" if graphs else "eager") +
                              (", 1 stream" if side is None else
                               ", 2 streams (dX||dW" + (")" if grouped else ", x||W quantize)")) +
-                             (", all W + first x quantized in one grouped launch" if grouped else ""),
+                             (", all W + first x quantized in one grouped launch" if grouped else "") +
+                             (f", GEMMs split {stack.split_k} ways along K" if stack.split_k > 1 else ""),
                    "launches_per_step": stack.launches_per_step(grouped),
                    "order": "forward over linears, then backward in reverse",
                    "parallelism": f"replicas x{world}"},
@@ -709,8 +731,10 @@ def run_kernel(args):
             sets.append((a, b))
         sa = torch.ones(1, device="cuda")
         out = torch.empty(M * N, dtype=torch.bfloat16, device="cuda")
-        call = lambda i: fp8.fp8_mm(sets[i % 2][0], E4M3, sets[i % 2][1], E4M3, sa, sa, layout, M, N, K, 1, 0, 0, 0,
-                                    None, None, 0, out, stream=st)
+        need = fp8.fp8_mm_workspace_size(M, N, K, 1, layout, args.split_k)
+        ws = torch.zeros(max(need, 4096), dtype=torch.uint8, device="cuda") if need else None
+        call = lambda i: fp8.fp8_mm_ws(sets[i % 2][0], E4M3, sets[i % 2][1], E4M3, sa, sa, layout, M, N, K, 1, 0, 0,
+                                       0, None, None, 0, out, ws, args.split_k if need else 0, stream=st)
         units = 2.0 * M * N * K
     else:
         n = int(args.shape)
@@ -757,6 +781,7 @@ def main():
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--one-stream", action="store_true", help="issue the whole step on one stream")
     ap.add_argument("--no-grouped", action="store_true", help="quantize every tensor with its own launch")
+    ap.add_argument("--split-k", type=int, default=0, help="force this many K splits in the GEMMs (0: library choice)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-compare", action="store_true", help="skip the bf16 / autograd comparison")

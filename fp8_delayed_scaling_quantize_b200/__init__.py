@@ -68,6 +68,9 @@ def _load():
         "fp8_selftest_wait_timeout": (I, [ctypes.c_uint32, P]),
         "fp8_bias_grad": (I, [P, I64, I64, P, P]),
         "fp8_quantize_many": (I, [P, ctypes.c_int32, P]),
+        "fp8_mm_ws": (I, [P, I, P, I, P, P, I, I64, I64, I64, I64, I64, I64, I64, P, P, I, P, P, ctypes.c_size_t,
+                          ctypes.c_int32, P]),
+        "fp8_mm_workspace_size": (ctypes.c_size_t, [I64, I64, I64, I64, I, ctypes.c_int32]),
     }
     for name, (res, args) in sig.items():
         try:
@@ -149,6 +152,22 @@ def fp8_mm(a8, fa, b8, fb, sa, sb, layout, M, N, K, batch, stride_a, stride_b, s
                              int(M), int(N), int(K), int(batch), int(stride_a), int(stride_b),
                              int(stride_c), _ptr(bias), _ptr(bias_scale), int(bias_fmt), _ptr(out),
                              _stream(stream)), "fp8_mm")
+
+
+def fp8_mm_ws(a8, fa, b8, fb, sa, sb, layout, M, N, K, batch, stride_a, stride_b, stride_c, bias,
+              bias_scale, bias_fmt, out, workspace, split_k=0, workspace_bytes=None, stream=None):
+    """fp8_mm that splits K `split_k` ways using `workspace` (a
+    zero-initialised device buffer; its size defaults to the tensor's nbytes)."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    return _check(lib.fp8_mm_ws(_ptr(a8), int(fa), _ptr(b8), int(fb), _ptr(sa), _ptr(sb), int(layout),
+                                int(M), int(N), int(K), int(batch), int(stride_a), int(stride_b),
+                                int(stride_c), _ptr(bias), _ptr(bias_scale), int(bias_fmt), _ptr(out),
+                                _ptr(workspace), int(workspace_bytes), int(split_k), _stream(stream)), "fp8_mm_ws")
+
+
+def fp8_mm_workspace_size(M, N, K, batch, layout, split_k):
+    return int(lib.fp8_mm_workspace_size(int(M), int(N), int(K), int(batch), int(layout), int(split_k)))
 
 
 def fp8_last_device_error():

@@ -14,7 +14,8 @@
 //    BM x BN = 128 x {64,128,256} in M-fastest order so CTAs that run together
 //    share the B (weight) tile in L2;
 //  * 6 warps with fixed roles: warp 0 issues TMA loads (one lane), warp 1
-//    owns TMEM and issues tcgen05.mma (one lane), warps 2-5 run the epilogue;
+//    owns TMEM and issues tcgen05.mma (one lane), warps 2-5 run the epilogue
+//    (one per TMEM lane quarter);
 //  * operands arrive by TMA in 128-byte-swizzled shared-memory stages of
 //    BK = 128 bytes of K, in their stored orientation: K-major for A in
 //    NT/NN and B in NT, MN-major for A in TN and B in NN/TN (the tensor core
@@ -25,8 +26,12 @@
 //  * two TMEM accumulators (2 x BN columns): the epilogue of tile i overlaps
 //    the main loop of tile i+1;
 //  * epilogue: tcgen05.ld 32 columns at a time, y = acc * (1/sa)(1/sb) +
-//    bias in fp32 (one fma), one round-to-nearest-even to bf16, guarded
-//    stores (exact M / N tails);
+//    bias in fp32 (one fma), one round-to-nearest-even to bf16, staged as
+//    128 x 32 tiles in shared memory and written by one TMA store each (TMA
+//    clips the M / N tails);
+//  * split K (with a caller workspace): a tile's k-blocks are shared by
+//    several CTAs; the last to finish adds the others' fp32 partials in split
+//    order and runs the epilogue;
 //  * every mbarrier wait is bounded by a time limit; a wait that gives up
 //    records FP8_ERR_DEVICE_TIMEOUT in the library's device error word and the
 //    CTA stops issuing work and exits through the normal teardown.
@@ -51,7 +56,8 @@ using namespace sm100;
 
 constexpr int BM = 128;
 constexpr int BK = 128;  // bytes = elements of K per stage
-constexpr int kThreads = 192;
+constexpr int kEpiThreads = 128;            // 4 epilogue warps, one per TMEM lane quarter
+constexpr int kThreads = 64 + kEpiThreads;  // producer warp, MMA warp, epilogue
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
 struct GemmParams {
@@ -70,6 +76,10 @@ struct GemmParams {
     int64_t stride_c;
     int vec_store;  // 16-byte stores allowed (N, stride_c multiples of 8, base aligned)
     int tma_store;  // tiles leave through shared memory and TMA stores (same conditions)
+    // split K: every tile is `split` work units of up to kb_per k-blocks each
+    int split, kb_per, total_units;
+    float* ws;         // fp32 partial slots: [tile][rank][split] x (128 x BN)
+    uint32_t* ws_cnt;  // per (tile, rank): {units arrived, partials written}
 };
 
 // Wait for phase `parity` of the mbarrier at `bar`, giving up after
@@ -80,6 +90,31 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 1023u) == 0 && globaltimer_ns() - t0 > limit_ns) {
+            atomicOr(&g_device_error, 1u);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* ptr) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void red_release_add(uint32_t* ptr, uint32_t v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
+}
+
+// Wait until the counter at `ptr` reaches `want`, giving up (device error
+// word set, false returned) after `limit_ns`.
+__device__ __forceinline__ bool wait_count(const uint32_t* ptr, uint32_t want, uint64_t limit_ns = kWaitLimitNs) {
+    if (ld_acquire_u32(ptr) >= want) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        __nanosleep(32);
+        if (ld_acquire_u32(ptr) >= want) return true;
+        if ((i & 255u) == 0 && globaltimer_ns() - t0 > limit_ns) {
             atomicOr(&g_device_error, 1u);
             return false;
         }
@@ -122,15 +157,24 @@ struct Smem {
     static constexpr int kBBytes = (BN / CTAS) * BK;
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kStageTx = CTAS * kStageBytes;  // bytes landing on the leader's full barrier
-    // per epilogue warp, two 32x32 bf16 staging buffers (64-byte swizzle)
-    static constexpr int kStgBufBytes = 32 * 32 * 2;
-    static constexpr int kStgOffset = STAGES * kStageBytes;
-    static constexpr int kBiasOffset = kStgOffset + 4 * 2 * kStgBufBytes;  // BN fp32 bias values
+    // two 128-row x 32-column bf16 staging tiles (64-byte swizzle), used in
+    // turn; 16 KB in all, so that a waiting kernel's small blocks still fit
+    // on the SM beside this CTA
+    static constexpr int kStgBytes = BM * 32 * 2;
+    static constexpr int kStgOffset = STAGES * kStageBytes;  // a multiple of 1024
+    static constexpr int kBiasOffset = kStgOffset + 2 * kStgBytes;  // BN fp32 bias values
     static constexpr int kBarOffset = kBiasOffset + BN * 4;
-    // full[S], empty[S], tmem_full[2], tmem_empty[2], then the TMEM slot
+    // full[S], empty[S], tmem_full[2], tmem_empty[2], then the TMEM slot and the split ticket
     static constexpr int kBytes = kBarOffset + (2 * STAGES + 4) * 8 + 16;
     static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024
     static constexpr uint32_t kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;
+    static_assert(kStgOffset % 1024 == 0, "staging tiles need 1024-byte alignment");
+    static_assert(kAlloc <= 227 * 1024, "shared memory per CTA");
+};
+
+// The tile walk's scalars, read once into registers.
+struct TileWalk {
+    int m_tiles, n_tiles, group_m;
 };
 
 // Tile order: batch outermost; inside a batch, groups of `group_m` M-tile
@@ -138,22 +182,43 @@ struct Smem {
 // running tiles then covers a compact block of rows and columns whose A and B
 // panels stay resident in L2 (an M-fastest walk over all rows streams the
 // whole A through L2 every wave).
-__device__ __forceinline__ void tile_coords(int t, const GemmParams& p, int& mb, int& nb, int& b) {
-    const int per_batch = p.m_tiles * p.n_tiles;
+__device__ __forceinline__ void tile_coords(int t, const TileWalk& w, int& mb, int& nb, int& b) {
+    const int per_batch = w.m_tiles * w.n_tiles;
     b = t / per_batch;
     const int r = t - b * per_batch;
-    const int per_group = p.group_m * p.n_tiles;
+    const int per_group = w.group_m * w.n_tiles;
     const int g = r / per_group;
-    const int first_m = g * p.group_m;
-    const int rows = min(p.group_m, p.m_tiles - first_m);
+    const int first_m = g * w.group_m;
+    const int rows = min(w.group_m, w.m_tiles - first_m);
     const int i = r - g * per_group;
     mb = first_m + i % rows;
     nb = i / rows;
 }
 
-__device__ __forceinline__ void epilogue_bar() {
-    // named barrier 1 over the 4 epilogue warps (128 threads)
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+// Keeps a value's computation (a kernel-parameter read) at this point of the
+// program: the first read of each parameter is a slow constant-cache miss, so
+// the kernel issues them all together while its set-up runs.
+template <typename T>
+__device__ __forceinline__ T pin(T v) {
+    asm volatile("" : "+r"(v));
+    return v;
+}
+
+// Named barrier 1: the epilogue warps.
+__device__ __forceinline__ void epilogue_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory"); }
+
+// Barrier 1, returning whether any epilogue thread passed true.
+__device__ __forceinline__ bool epilogue_bar_or(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred q, p;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.or.pred p, 1, %2, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"(uint32_t(v)), "n"(kEpiThreads)
+        : "memory");
+    return r != 0;
 }
 
 // One kernel for both tile shapes: CTAS = 1 computes 128 x BN tiles per CTA;
@@ -161,8 +226,12 @@ __device__ __forceinline__ void epilogue_bar() {
 // with tcgen05 cta_group::2 -- the leader issues the MMAs, each CTA loads its
 // own 128 rows of A and BN/2 columns of B (halving each SM's operand
 // traffic) and writes its own 128 output rows.
-template <int BN, bool A_MN, bool B_MN, int STAGES, bool HAS_BIAS, int CTAS>
-__global__ void __launch_bounds__(kThreads, 1)
+//
+// Epilogue: 4 warps, one per TMEM lane quarter. Every 32 columns of the tile
+// become a 128 x 32 bf16 tile in shared memory that one thread writes with a
+// single TMA store (8 stores for a 128 x 256 tile).
+template <int BN, bool A_MN, bool B_MN, int STAGES, bool HAS_BIAS, int CTAS, bool SPLIT>
+__global__ void __maxnreg__(168)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const __grid_constant__ CUtensorMap tm_c, const GemmParams p) {
     using L = Smem<BN, STAGES, CTAS>;
@@ -177,14 +246,26 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     const uint32_t bar_tfull = bar_empty + STAGES * 8;
     const uint32_t bar_tempty = bar_tfull + 2 * 8;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBarOffset + (2 * STAGES + 4) * 8);
+    uint32_t* ticket_slot = tmem_slot + 1;  // split K: the epilogue's arrival ticket
     float* s_bias = reinterpret_cast<float*>(smem + L::kBiasOffset);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const uint32_t rank = CTAS == 2 ? cluster_ctarank() : 0u;  // 0 = the pair's leader
     const bool leader = rank == 0;
-    const int unit0 = blockIdx.x / CTAS;     // this CTA's first tile (a pair shares it)
-    const int unit_step = gridDim.x / CTAS;  // tiles advance by the number of CTAs (pairs)
+    const int unit0 = blockIdx.x / CTAS;     // this CTA's first work unit (a pair shares it)
+    const int unit_step = gridDim.x / CTAS;  // units advance by the number of CTAs (pairs)
+
+    // every parameter the roles read, fetched together now
+    const int total_units = pin(p.total_units);
+    const int k_blocks = pin(p.k_blocks);
+    const int split = SPLIT ? pin(p.split) : 1;  // without SPLIT the split-K code compiles away
+    const int kb_per = SPLIT ? pin(p.kb_per) : k_blocks;
+    const TileWalk walk = {pin(p.m_tiles), pin(p.n_tiles), pin(p.group_m)};
+    const int a_bcast = pin(p.a_bcast), b_bcast = pin(p.b_bcast);
+    const uint32_t idesc = pin(p.idesc);
+    const int M = pin(p.M), N = pin(p.N);
+    const int tma_store = pin(p.tma_store), vec_store = pin(p.vec_store);
 
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -193,12 +274,12 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar_tfull + 8 * b, 1);
-            mbar_init(bar_tempty + 8 * b, CTAS * 4 * 32);
+            mbar_init(bar_tempty + 8 * b, CTAS * kEpiThreads);
         }
         fence_mbar_init();
         tma_prefetch(&tm_a);
         tma_prefetch(&tm_b);
-        if (p.tma_store) tma_prefetch(&tm_c);
+        if (tma_store) tma_prefetch(&tm_c);
     }
     if (warp == 1) {
         tmem_alloc<CTAS>(smem_addr(tmem_slot), L::kTmemCols);
@@ -220,14 +301,17 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int t = unit0; t < p.total_tiles && ok; t += unit_step) {
+            for (int u = unit0; u < total_units && ok; u += unit_step) {
+                const int t = u / split;
+                const int kb0 = (u - t * split) * kb_per;
+                const int kb1 = min(k_blocks, kb0 + kb_per);
                 int mb, nb, b;
-                tile_coords(t, p, mb, nb, b);
-                const int ba = p.a_bcast ? 0 : b;
-                const int bb = p.b_bcast ? 0 : b;
+                tile_coords(t, walk, mb, nb, b);
+                const int ba = a_bcast ? 0 : b;
+                const int bb = b_bcast ? 0 : b;
                 const int m0 = mb * BM * CTAS + int(rank) * BM;
                 const int n0 = nb * BN + int(rank) * (BN / CTAS);
-                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!wait_bounded(bar_empty + 8 * stage, phase ^ 1)) { ok = false; break; }
                     const uint32_t full = bar_full + 8 * stage;
                     if (leader) mbar_arrive_expect_tx(full, L::kStageTx);
@@ -266,13 +350,16 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             uint32_t phase = 0;
             int it = 0;
             bool ok = true;
-            for (int t = unit0; t < p.total_tiles && ok; t += unit_step, ++it) {
+            for (int u = unit0; u < total_units && ok; u += unit_step, ++it) {
+                const int t = u / split;
+                const int kb0 = (u - t * split) * kb_per;
+                const int kb1 = min(k_blocks, kb0 + kb_per);
                 const int buf = it & 1;
                 const uint32_t acc_phase = (it >> 1) & 1;
                 if (!wait_bounded(bar_tempty + 8 * buf, acc_phase ^ 1)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + buf * BN;
-                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!wait_bounded(bar_full + 8 * stage, phase)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t da = s_a + stage * L::kABytes;
@@ -285,7 +372,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                                                     : smem_desc_sw128(da + j * 32, 16, 1024);
                         const uint64_t bdesc = B_MN ? smem_desc_sw128(db + j * 32 * 128, 128 * BK, 1024)
                                                     : smem_desc_sw128(db + j * 32, 16, 1024);
-                        mma_f8f6f4<CTAS>(d_tmem, adesc, bdesc, p.idesc, (kb | j) != 0);
+                        mma_f8f6f4<CTAS>(d_tmem, adesc, bdesc, idesc, kb != kb0 || j != 0);
                     }
                     // release the stage (in both CTAs of a pair)
                     if (CTAS == 1) mma_commit(bar_empty + 8 * stage);
@@ -298,28 +385,31 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         }
     } else {
         // ----------------------------------------------------- epilogue ---
-        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int q = warp & 3;             // TMEM lane quarter this warp may access
         const int row_in_tile = q * 32 + lane;
-        const int etid = threadIdx.x - 64;  // 0..127 over the epilogue warps
+        const int etid = threadIdx.x - 64;  // 0 .. kEpiThreads-1
+        const bool store_lead = etid == 0;  // issues the TMA stores
+        const uint32_t stg0 = s_base + L::kStgOffset;
+        int n_st = 0;  // TMA stores issued so far (they alternate between the two staging tiles)
         const float inv = (1.0f / __ldg(p.sa)) * (1.0f / __ldg(p.sb));
         const float bscale = (HAS_BIAS && p.bias_kind == 2) ? __ldg(p.bias_scale) : 1.0f;
-        const uint32_t s_stg = s_base + L::kStgOffset;
-        int stg_n = 0;  // TMA stores issued by this warp
         bool failed = false;
         int it = 0;
-        for (int t = unit0; t < p.total_tiles; t += unit_step, ++it) {
+        for (int u = unit0; u < total_units; u += unit_step, ++it) {
+            const int t = u / split;
+            const int split_id = u - t * split;
             int mb, nb, b;
-            tile_coords(t, p, mb, nb, b);
+            tile_coords(t, walk, mb, nb, b);
             const int buf = it & 1;
             const uint32_t acc_phase = (it >> 1) & 1;
             const int m0 = mb * BM * CTAS + int(rank) * BM;  // this CTA's first output row
             if (HAS_BIAS) {
                 // the tile's BN bias values, dequantized once into shared memory
                 epilogue_bar();  // the previous tile's readers are done
-                for (int j = etid; j < BN; j += 128) {
+                for (int j = etid; j < BN; j += kEpiThreads) {
                     const int col = nb * BN + j;
                     float v = 0.0f;
-                    if (col < p.N) {
+                    if (col < N) {
                         if (p.bias_kind == 1) {
                             v = __uint_as_float(uint32_t(__ldg(static_cast<const uint16_t*>(p.bias) + col)) << 16);
                         } else {
@@ -331,77 +421,142 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                 }
                 epilogue_bar();
             }
-            // every lane waits, then the warp agrees (and reconverges) before
-            // the warp-collective TMEM loads. After a wait gave up, the warp
-            // keeps walking the tiles without waiting so that the epilogue
-            // warps still meet at every named barrier above.
-            if (!failed) {
-                const bool ok = wait_bounded(bar_tfull + 8 * buf, acc_phase);
-                failed = !__all_sync(0xffffffffu, ok);
-            }
+            // every lane waits, then all epilogue warps agree (and each warp
+            // reconverges) before the warp-collective TMEM loads. After a wait
+            // gave up, they all keep walking the units without waiting, so that
+            // they still meet at every named barrier.
+            if (!failed) failed = !wait_bounded(bar_tfull + 8 * buf, acc_phase);
+            failed = epilogue_bar_or(failed);
             if (failed) continue;
             tc_fence_after();
+            const uint32_t t_row = tmem_base + (uint32_t(q * 32) << 16) + buf * BN;
+            // Split K: the unit that arrives last at its tile finishes it; the
+            // others leave their fp32 partial in the workspace. Slot layout:
+            // 16-byte piece v of 32-column chunk c of tile row r sits at
+            // ((c * 8 + v) * 128 + r) * 16, so each store and load instruction
+            // of a warp covers 512 contiguous bytes.
+            const float4* slots = nullptr;
+            if (SPLIT && split > 1) {
+                uint32_t* cnt = p.ws_cnt + 2 * (t * CTAS + int(rank));
+                slots = reinterpret_cast<const float4*>(p.ws) + size_t(t * CTAS + int(rank)) * split * (BM * BN / 4);
+                if (etid == 0) *ticket_slot = atomicAdd(cnt, 1u);
+                epilogue_bar();
+                const bool last = *ticket_slot == uint32_t(split - 1);
+                if (!last) {
+                    float4* mine = const_cast<float4*>(slots) + size_t(split_id) * (BM * BN / 4);
+#pragma unroll 1
+                    for (int c = 0; c < BN / 32; ++c) {
+                        if (nb * BN + c * 32 >= N) break;  // uniform; the finisher skips it too
+                        uint32_t r[32];
+                        tmem_ld32(t_row + c * 32, r);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int v = 0; v < 8; ++v)
+                            __stcg(mine + (c * 8 + v) * 128 + row_in_tile,
+                                   make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                               __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])));
+                    }
+                    __threadfence();
+                    epilogue_bar();
+                    if (etid == 0) red_release_add(cnt + 1, 1u);
+                    tc_fence_before();
+                    if (CTAS == 1) mbar_arrive(bar_tempty + 8 * buf);
+                    else           mbar_arrive_cluster(map_to_rank(bar_tempty + 8 * buf, 0));
+                    continue;
+                }
+                if (etid == 0) {
+                    wait_count(cnt + 1, uint32_t(split - 1));
+                    cnt[0] = 0u;  // the tile's counters are ready for the next call
+                    cnt[1] = 0u;
+                }
+                epilogue_bar();
+            }
             const int row = m0 + row_in_tile;
-            uint16_t* orow = p.out + int64_t(b) * p.stride_c + int64_t(row) * p.N;
+            uint16_t* orow = p.out + int64_t(b) * p.stride_c + int64_t(row) * N;
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tmem_base + (uint32_t(q * 32) << 16) + buf * BN + c * 32, r);
-                tmem_ld_wait();
                 const int col0 = nb * BN + c * 32;
-                if (col0 >= p.N) continue;                       // warp-uniform
-                if (!p.tma_store && row >= p.M) continue;
+                if (col0 >= N) break;  // uniform over the epilogue warps
+                uint32_t r[32];
+                tmem_ld32(t_row + c * 32, r);
+                tmem_ld_wait();
+                if (SPLIT && split > 1) {
+                    // the sum over the splits in split order, whatever order
+                    // they arrived in (the result does not depend on timing)
+                    float acc[32];
+#pragma unroll 1
+                    for (int sp = 0; sp < split; ++sp) {
+                        if (sp == split_id) {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                acc[i] = sp == 0 ? __uint_as_float(r[i]) : acc[i] + __uint_as_float(r[i]);
+                        } else {
+                            const float4* src = slots + size_t(sp) * (BM * BN / 4) + c * 8 * 128 + row_in_tile;
+#pragma unroll
+                            for (int v = 0; v < 8; ++v) {
+                                const float4 x = __ldcg(src + v * 128);
+                                acc[4 * v] = sp == 0 ? x.x : acc[4 * v] + x.x;
+                                acc[4 * v + 1] = sp == 0 ? x.y : acc[4 * v + 1] + x.y;
+                                acc[4 * v + 2] = sp == 0 ? x.z : acc[4 * v + 2] + x.z;
+                                acc[4 * v + 3] = sp == 0 ? x.w : acc[4 * v + 3] + x.w;
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(acc[i]);
+                }
                 float y[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const float bias = HAS_BIAS ? s_bias[c * 32 + i] : 0.0f;
                     y[i] = fmaf(__uint_as_float(r[i]), inv, bias);
                 }
-                if (p.tma_store) {
-                    // stage the warp's 32 x 32 bf16 block (64-byte swizzle: the
-                    // 16-byte chunk index XOR (row / 2) mod 4 keeps the 8 lanes of
-                    // a store phase on distinct banks), then one TMA store; it
-                    // clips the M / N tails of the output
-                    const uint32_t stg = s_stg + (q * 2 + (stg_n & 1)) * L::kStgBufBytes;
-                    if (stg_n >= 2) {
-                        if (lane == 0) bulk_wait_read<1>();
-                        __syncwarp();
-                    }
+                if (tma_store) {
+                    // the 128 x 32 bf16 block goes to the staging tile whose last
+                    // store is known to have read it (64-byte swizzle: 16-byte
+                    // piece j of row r at (j ^ (r / 2 mod 4)) * 16, so the 8
+                    // lanes of a store phase hit distinct banks); then one TMA
+                    // store, which clips the M / N tails of the output
+                    const uint32_t stg = stg0 + (n_st & 1) * L::kStgBytes;
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        const uint32_t w0 = pack_bf16x2(y[8 * j + 0], y[8 * j + 1]);
-                        const uint32_t w1 = pack_bf16x2(y[8 * j + 2], y[8 * j + 3]);
-                        const uint32_t w2 = pack_bf16x2(y[8 * j + 4], y[8 * j + 5]);
-                        const uint32_t w3 = pack_bf16x2(y[8 * j + 6], y[8 * j + 7]);
-                        const uint32_t addr = stg + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4);
-                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w0), "r"(w1),
-                                     "r"(w2), "r"(w3)
+                        const uint32_t addr = stg + row_in_tile * 64 + ((j ^ ((row_in_tile >> 1) & 3)) << 4);
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                                     "r"(pack_bf16x2(y[8 * j + 0], y[8 * j + 1])),
+                                     "r"(pack_bf16x2(y[8 * j + 2], y[8 * j + 3])),
+                                     "r"(pack_bf16x2(y[8 * j + 4], y[8 * j + 5])),
+                                     "r"(pack_bf16x2(y[8 * j + 6], y[8 * j + 7]))
                                      : "memory");
                     }
                     fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_3d(&tm_c, stg, col0, m0 + q * 32, b);
+                    // the previous store has read the other tile, which the next
+                    // block reuses; the barrier publishes that and this block
+                    if (store_lead) bulk_wait_read<0>();
+                    epilogue_bar();
+                    if (store_lead) {
+                        tma_store_3d(&tm_c, stg, col0, m0, b);
                         bulk_commit();
                     }
-                    ++stg_n;
-                } else if (p.vec_store && col0 + 32 <= p.N) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + col0);
+                    ++n_st;
+                } else if (row < M) {
+                    if (vec_store && col0 + 32 <= N) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + col0);
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        uint4 w;
-                        w.x = pack_bf16x2(y[8 * v + 0], y[8 * v + 1]);
-                        w.y = pack_bf16x2(y[8 * v + 2], y[8 * v + 3]);
-                        w.z = pack_bf16x2(y[8 * v + 4], y[8 * v + 5]);
-                        w.w = pack_bf16x2(y[8 * v + 6], y[8 * v + 7]);
-                        dst[v] = w;
-                    }
-                } else {
+                        for (int v = 0; v < 4; ++v) {
+                            uint4 x;
+                            x.x = pack_bf16x2(y[8 * v + 0], y[8 * v + 1]);
+                            x.y = pack_bf16x2(y[8 * v + 2], y[8 * v + 3]);
+                            x.z = pack_bf16x2(y[8 * v + 4], y[8 * v + 5]);
+                            x.w = pack_bf16x2(y[8 * v + 6], y[8 * v + 7]);
+                            dst[v] = x;
+                        }
+                    } else {
 #pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        const uint32_t w = pack_bf16x2(y[i], y[i + 1]);
-                        if (col0 + i < p.N) orow[col0 + i] = uint16_t(w & 0xFFFFu);
-                        if (col0 + i + 1 < p.N) orow[col0 + i + 1] = uint16_t(w >> 16);
+                        for (int i = 0; i < 32; i += 2) {
+                            const uint32_t x = pack_bf16x2(y[i], y[i + 1]);
+                            if (col0 + i < N) orow[col0 + i] = uint16_t(x & 0xFFFFu);
+                            if (col0 + i + 1 < N) orow[col0 + i + 1] = uint16_t(x >> 16);
+                        }
                     }
                 }
             }
@@ -410,9 +565,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             if (CTAS == 1) mbar_arrive(bar_tempty + 8 * buf);
             else           mbar_arrive_cluster(map_to_rank(bar_tempty + 8 * buf, 0));
         }
-        // the staging buffers must outlive the stores that read them, and the
-        // output must be complete when the grid is
-        if (p.tma_store && lane == 0) bulk_wait_all();
+        // the staging tiles must outlive the stores that read them; the global
+        // writes themselves complete with the grid (a dependent kernel's
+        // griddepcontrol.wait and stream order both see them)
+        if (tma_store && store_lead) bulk_wait_read<0>();
     }
 
     tc_fence_before();
@@ -465,8 +621,8 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 3-D map over the bf16 output (N, M, batch), 32 x 32 boxes with a 64-byte
-// swizzle matching the epilogue's staging layout.
+// 3-D map over the bf16 output (N, M, batch), 32-column x 128-row boxes with
+// a 64-byte swizzle matching the epilogue's staging tiles.
 bool make_out_map(CUtensorMap* map, void* base, uint64_t n, uint64_t m, uint64_t batch, uint64_t batch_stride_bytes) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
@@ -476,7 +632,7 @@ bool make_out_map(CUtensorMap* map, void* base, uint64_t n, uint64_t m, uint64_t
     }
     cuuint64_t dims[3] = {n, m, batch};
     cuuint64_t strides[2] = {n * 2, batch_stride_bytes};
-    cuuint32_t box[3] = {32, 32, 1};
+    cuuint32_t box[3] = {32, uint32_t(BM), 1};
     cuuint32_t estr[3] = {1, 1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
               CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
@@ -501,11 +657,11 @@ struct HostArgs {
     int64_t batch, stride_b;
 };
 
-template <int BN, bool A_MN, bool B_MN, int STAGES, bool HAS_BIAS, int CTAS>
+template <int BN, bool A_MN, bool B_MN, int STAGES, bool HAS_BIAS, int CTAS, bool SPLIT>
 fp8_status launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, GemmParams p,
                       const HostArgs& h, cudaStream_t st) {
     using L = Smem<BN, STAGES, CTAS>;
-    auto kern = fp8_gemm_kernel<BN, A_MN, B_MN, STAGES, HAS_BIAS, CTAS>;
+    auto kern = fp8_gemm_kernel<BN, A_MN, B_MN, STAGES, HAS_BIAS, CTAS, SPLIT>;
     static bool attr_set[64] = {false};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8_ERR_CUDA;
@@ -520,8 +676,11 @@ fp8_status launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
     const int64_t tiles = int64_t(p.m_tiles) * p.n_tiles * h.batch;
     p.total_tiles = int(tiles);
     p.group_m = CTAS == 2 ? 8 : 16;  // about sqrt(concurrent tiles) rows per group
+    p.kb_per = (p.k_blocks + p.split - 1) / p.split;
+    const int64_t work = tiles * p.split;
+    p.total_units = int(work);
     const int64_t units_max = sm_count() / CTAS;
-    const int units = int(tiles < units_max ? tiles : units_max);
+    const int units = int(work < units_max ? work : units_max);
     return launch_pdl(kern, units * CTAS, kThreads, L::kAlloc, st, CTAS, ta, tb, tc, p);
 }
 
@@ -529,48 +688,90 @@ template <int BN, bool A_MN, bool B_MN, int STAGES, int CTAS>
 fp8_status launch(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, const HostArgs& h, cudaStream_t st) {
     CUtensorMap tc = {};
     if (p.tma_store && !make_out_map(&tc, p.out, p.N, p.M, h.batch, uint64_t(p.stride_c) * 2)) return FP8_ERR_CUDA;
-    return p.bias_kind ? launch_one<BN, A_MN, B_MN, STAGES, true, CTAS>(ta, tb, tc, p, h, st)
-                       : launch_one<BN, A_MN, B_MN, STAGES, false, CTAS>(ta, tb, tc, p, h, st);
+    if (p.split > 1)
+        return p.bias_kind ? launch_one<BN, A_MN, B_MN, STAGES, true, CTAS, true>(ta, tb, tc, p, h, st)
+                           : launch_one<BN, A_MN, B_MN, STAGES, false, CTAS, true>(ta, tb, tc, p, h, st);
+    return p.bias_kind ? launch_one<BN, A_MN, B_MN, STAGES, true, CTAS, false>(ta, tb, tc, p, h, st)
+                       : launch_one<BN, A_MN, B_MN, STAGES, false, CTAS, false>(ta, tb, tc, p, h, st);
 }
 
 // Tile choice for 148 SMs by a small cost model: a persistent grid walks
-// ceil(tiles / CTAs) rounds of tiles, each costing k_blocks times the
-// per-k-block time of that tile shape, plus the one epilogue left exposed at
-// the end. The per-k-block times (microseconds at the clocks seen under load)
-// and epilogue times were measured on B200 with this kernel: 128x256 0.48,
-// 128x128 0.40, 128x64 0.30, an SM pair's 256x256 0.43. Pairs are used only
-// with at least one 256x256 tile per SM (below that their coarser grain
-// loses). MN-major B needs whole 128-byte swizzle atoms along N per CTA.
+// ceil(units / CTAs) rounds of work units, each costing its k-blocks times
+// the per-k-block time of that tile shape, plus the one epilogue left exposed
+// at the end. The per-k-block times (microseconds at the clocks seen under
+// load) and epilogue times were measured on B200 with this kernel: 128x256
+// 0.48, 128x128 0.40, 128x64 0.30, an SM pair's 256x256 0.43 and 256x128
+// 0.25. An SM pair's 256 x 128 tile loads 24 KB per SM per k-block, so eight
+// stages keep its MMAs fed; a single SM's 128 x 128 tile needs 32 KB per
+// k-block for half the MMA work and waits on its loads. Pairs of 256 x 256
+// are used only with at least one such tile per SM (below that their coarser
+// grain loses). MN-major B needs whole 128-byte swizzle atoms along N per
+// CTA, so the 256 x 128 pair tile takes K-major B only.
+//
+// Split K (split_req >= 2, with a workspace): a tile becomes `split` units
+// over consecutive k-block ranges; the unit that finishes last adds the
+// others' fp32 partials and runs the epilogue. The automatic choice
+// (split_req = 0) does not split: on every shape measured on B200 the
+// partials' round trip through L2 cost more than the shorter main loop saved.
+constexpr size_t kSplitCntBytes = 4096;  // two counters per (tile, CTA of the tile)
+constexpr int kMaxSplit = 4;
+
 struct TileChoice {
     bool pair;
     int bn;
+    int split;  // 0: the requested split is not possible for this problem
 };
 
-inline TileChoice choose_tile(int64_t M, int64_t N, int64_t K, int64_t batch, bool b_mn, int64_t sms) {
+inline size_t split_ws_bytes(int64_t tiles, int ctas, int bn, int split) {
+    return kSplitCntBytes + size_t(tiles) * ctas * split * BM * bn * sizeof(float);
+}
+
+inline int64_t tile_count(int64_t M, int64_t N, int64_t batch, bool pair, int bn) {
+    const int64_t rows = BM * (pair ? 2 : 1);
+    return ((M + rows - 1) / rows) * ((N + bn - 1) / bn) * batch;
+}
+
+inline TileChoice choose_tile(int64_t M, int64_t N, int64_t K, int64_t batch, bool b_mn, int64_t sms,
+                              int split_req) {
     const int64_t kb = (K + BK - 1) / BK;
-    auto cost = [&](int64_t rows, int bn, int64_t units, double t_k, double t_epi) {
-        const int64_t tiles = ((M + rows - 1) / rows) * ((N + bn - 1) / bn) * batch;
-        const int64_t rounds = (tiles + units - 1) / units;
-        return double(rounds) * double(kb) * t_k + t_epi;
+    const int split = split_req < 2 ? 1 : split_req;
+    const int64_t kb_per = (kb + split - 1) / split;
+    if (split > 1 && (split - 1) * kb_per >= kb) return {false, 256, 0};  // every unit needs k-blocks
+    auto cost = [&](bool pair, int bn, double t_k, double t_epi) {
+        const int ctas = pair ? 2 : 1;
+        const int64_t units = sms / ctas;
+        const int64_t tiles = tile_count(M, N, batch, pair, bn);
+        if (split > 1 && size_t(tiles) * ctas * 2 * sizeof(uint32_t) > kSplitCntBytes) return 1e30;
+        const int64_t rounds = (tiles * split + units - 1) / units;
+        return double(rounds) * double(kb_per) * t_k + t_epi;
     };
-    const int64_t pair_tiles = ((M + 2 * BM - 1) / (2 * BM)) * ((N + 255) / 256) * batch;
-    if (M > BM && N > 128 && pair_tiles >= sms) return {true, 256};
-    TileChoice best = {false, 256};
-    double best_cost = cost(BM, 256, sms, 0.48, 2.0);
-    const double c128 = cost(BM, 128, sms, 0.40, 1.0);
-    if (c128 < best_cost) { best = {false, 128}; best_cost = c128; }
-    if (!b_mn) {
-        const double c64 = cost(BM, 64, sms, 0.30, 0.5);
-        if (c64 < best_cost) { best = {false, 64}; best_cost = c64; }
-    }
+    if (split == 1 && M > BM && N > 128 && tile_count(M, N, batch, true, 256) >= sms) return {true, 256, 1};
+    const bool pair_ok = M > BM;  // a pair's second CTA would hold only padding otherwise
+    const TileChoice c[4] = {{false, 256, split}, {false, 128, split}, {false, 64, split}, {true, 256, split}};
+    const double t[4] = {cost(false, 256, 0.48, 2.0), cost(false, 128, 0.40, 1.0),
+                         b_mn ? 1e30 : cost(false, 64, 0.30, 0.5),
+                         (split > 1 && pair_ok && N > 128) ? cost(true, 256, 0.43, 2.0) : 1e30};
+    TileChoice best = {false, 256, 0};
+    double best_cost = 1e30;
+    for (int i = 0; i < 4; ++i)
+        if (t[i] < best_cost) { best = c[i]; best_cost = t[i]; }
     return best;
 }
 
 template <bool A_MN, bool B_MN>
-fp8_status dispatch(const CUtensorMap& ta, GemmParams p, const HostArgs& h, cudaStream_t st) {
-    const TileChoice tc = choose_tile(p.M, p.N, p.K, h.batch, B_MN, sm_count());
+fp8_status dispatch(const CUtensorMap& ta, GemmParams p, const HostArgs& h, void* ws, size_t ws_bytes,
+                    int split_req, cudaStream_t st) {
+    const TileChoice tc = choose_tile(p.M, p.N, p.K, h.batch, B_MN, sm_count(), split_req);
+    if (tc.split == 0) return FP8_ERR_UNSUPPORTED;
     const bool pair = tc.pair;
     const int bn = tc.bn;
+    p.split = tc.split;
+    if (tc.split > 1) {
+        const int64_t tiles = tile_count(p.M, p.N, h.batch, pair, bn);
+        if (!ws || ws_bytes < split_ws_bytes(tiles, pair ? 2 : 1, bn, tc.split)) return FP8_ERR_INVALID_ARG;
+        p.ws_cnt = static_cast<uint32_t*>(ws);
+        p.ws = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kSplitCntBytes);
+    }
     CUtensorMap tb;
     const uint64_t sb_bytes = uint64_t(h.stride_b);
     const uint32_t b_box_n = pair ? bn / 2 : bn;  // N extent one CTA loads
@@ -589,10 +790,13 @@ fp8_status dispatch(const CUtensorMap& ta, GemmParams p, const HostArgs& h, cuda
 
 using namespace fp8lite;
 
-extern "C" fp8_status fp8_mm(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8, fp8_fmt fb, const float* sa,
-                             const float* sb, fp8_layout layout, int64_t M, int64_t N, int64_t K, int64_t batch,
-                             int64_t stride_a, int64_t stride_b, int64_t stride_c, const void* bias,
-                             const float* bias_scale, fp8_fmt bias_fmt, void* out, void* stream) {
+extern "C" fp8_status fp8_mm_ws(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8, fp8_fmt fb, const float* sa,
+                                const float* sb, fp8_layout layout, int64_t M, int64_t N, int64_t K, int64_t batch,
+                                int64_t stride_a, int64_t stride_b, int64_t stride_c, const void* bias,
+                                const float* bias_scale, fp8_fmt bias_fmt, void* out, void* workspace,
+                                size_t workspace_bytes, int32_t split_k, void* stream) {
+    if (split_k < 0 || split_k > kMaxSplit) return FP8_ERR_INVALID_ARG;
+    if (workspace && !aligned(workspace, 16)) return FP8_ERR_ALIGNMENT;
     if (!valid_fmt(fa) || !valid_fmt(fb)) return FP8_ERR_INVALID_ARG;
     if (layout != FP8_NT && layout != FP8_NN && layout != FP8_TN) return FP8_ERR_INVALID_ARG;
     if (!a8 || !b8 || !sa || !sb || !out) return FP8_ERR_INVALID_ARG;
@@ -634,6 +838,7 @@ extern "C" fp8_status fp8_mm(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8, f
     p.bias_fmt = bias_fmt;
     p.out = static_cast<uint16_t*>(out);
     p.stride_c = stride_c;
+    p.split = 1;
     p.vec_store = (N % 8 == 0) && (stride_c % 8 == 0) && aligned(out, 16);
     p.tma_store = p.vec_store;
 
@@ -644,10 +849,29 @@ extern "C" fp8_status fp8_mm(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8, f
     cudaStream_t st = as_stream(stream);
     const HostArgs h = {int(fa), int(fb), b8, batch, stride_b};
     switch (layout) {
-        case FP8_NT: return dispatch<false, false>(ta, p, h, st);
-        case FP8_NN: return dispatch<false, true>(ta, p, h, st);
-        default:     return dispatch<true, true>(ta, p, h, st);
+        case FP8_NT: return dispatch<false, false>(ta, p, h, workspace, workspace_bytes, split_k, st);
+        case FP8_NN: return dispatch<false, true>(ta, p, h, workspace, workspace_bytes, split_k, st);
+        default:     return dispatch<true, true>(ta, p, h, workspace, workspace_bytes, split_k, st);
     }
+}
+
+extern "C" fp8_status fp8_mm(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8, fp8_fmt fb, const float* sa,
+                             const float* sb, fp8_layout layout, int64_t M, int64_t N, int64_t K, int64_t batch,
+                             int64_t stride_a, int64_t stride_b, int64_t stride_c, const void* bias,
+                             const float* bias_scale, fp8_fmt bias_fmt, void* out, void* stream) {
+    return fp8_mm_ws(a8, fa, b8, fb, sa, sb, layout, M, N, K, batch, stride_a, stride_b, stride_c, bias, bias_scale,
+                     bias_fmt, out, nullptr, 0, 0, stream);
+}
+
+extern "C" size_t fp8_mm_workspace_size(int64_t M, int64_t N, int64_t K, int64_t batch, fp8_layout layout,
+                                        int32_t split_k) {
+    if (M < 1 || N < 1 || K < 1 || batch < 1 || split_k < 0 || split_k > kMaxSplit) return 0;
+    if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31) || batch >= (int64_t(1) << 31))
+        return 0;
+    if (layout != FP8_NT && layout != FP8_NN && layout != FP8_TN) return 0;
+    const TileChoice tc = choose_tile(M, N, K, batch, layout != FP8_NT, sm_count(), split_k);
+    if (tc.split < 2) return 0;
+    return split_ws_bytes(tile_count(M, N, batch, tc.pair, tc.bn), tc.pair ? 2 : 1, tc.bn, tc.split);
 }
 
 extern "C" fp8_status fp8_last_device_error(void) {

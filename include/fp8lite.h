@@ -189,6 +189,48 @@ FP8LITE_API fp8_status fp8_mm(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8, 
                   const void* bias, const float* bias_scale, fp8_fmt bias_fmt,
                   void* out, void* stream);
 
+/* fp8_mm that can split K over a caller-owned workspace: `split_k` CTAs (or
+ * SM pairs) share each output tile's k-blocks, each accumulating its part in
+ * fp32; the one that finishes last adds the others' partials in split order
+ * and runs the epilogue. The result is the same formula; only the fp32
+ * accumulation is grouped differently, so it stays within fp8_mm's accuracy,
+ * and it is deterministic: it does not depend on the order in which the
+ * splits finish.
+ *
+ * split_k         0: the library's choice (in this version: no split -- on
+ *                 every shape measured on B200 the partials' round trip
+ *                 through L2 cost more than the shorter main loop saved);
+ *                 1: no split; 2 .. 4: exactly that many splits.
+ * workspace       NULL when no split is requested, else device memory,
+ *                 16-byte aligned, of workspace_bytes >=
+ *                 fp8_mm_workspace_size(..., split_k) bytes. Its first 4096
+ *                 bytes are counters: they must be zero before the first call
+ *                 that uses the workspace (e.g. cudaMemsetAsync once after
+ *                 allocation), and every completed call leaves them zero
+ *                 again, so the workspace can be reused, also inside CUDA
+ *                 graphs. The rest holds fp32 partial tiles. The caller owns
+ *                 it; two calls that may run at the same time (e.g. on two
+ *                 streams) need two workspaces. After FP8_ERR_DEVICE_TIMEOUT
+ *                 it must be zeroed again.
+ * Other arguments and errors as fp8_mm, plus: FP8_ERR_INVALID_ARG for
+ * split_k outside 0..4 or a missing / too small workspace; FP8_ERR_UNSUPPORTED
+ * when the problem cannot take that split (fewer k-blocks of 128 than splits
+ * need, or more than 512 tile halves); FP8_ERR_ALIGNMENT for a misaligned
+ * workspace. */
+FP8LITE_API fp8_status fp8_mm_ws(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8, fp8_fmt fb,
+                  const float* sa, const float* sb, fp8_layout layout,
+                  int64_t M, int64_t N, int64_t K, int64_t batch,
+                  int64_t stride_a, int64_t stride_b, int64_t stride_c,
+                  const void* bias, const float* bias_scale, fp8_fmt bias_fmt,
+                  void* out, void* workspace, size_t workspace_bytes, int32_t split_k,
+                  void* stream);
+
+/* Workspace bytes fp8_mm_ws needs for this problem and split_k on the
+ * current device: 0 when that call would not split (split_k 0 or 1), or for
+ * arguments fp8_mm_ws rejects. */
+FP8LITE_API size_t fp8_mm_workspace_size(int64_t M, int64_t N, int64_t K, int64_t batch, fp8_layout layout,
+                                         int32_t split_k);
+
 /* Synchronises the current device, then reads and clears the library's
  * device error word: FP8_ERR_DEVICE_TIMEOUT if a GEMM thread block gave up a
  * bounded wait since the last call (its output tile is then undefined),

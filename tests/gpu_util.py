@@ -39,16 +39,26 @@ def codes(t):
 
 
 def mm(a8, fa, b8, fb, sa, sb, layout, M, N, K, batch=1, stride_a=None, stride_b=None,
-       stride_c=None, bias=None, bias_scale=None, bias_fmt=0, out=None):
-    """fp8_mm through the C ABI; allocates the bf16 output when not given."""
+       stride_c=None, bias=None, bias_scale=None, bias_fmt=0, out=None, ws=None, split_k=0):
+    """fp8_mm (fp8_mm_ws when a workspace is given) through the C ABI;
+    allocates the bf16 output when not given."""
     stride_a = M * K if stride_a is None else stride_a
     stride_b = N * K if stride_b is None else stride_b
     stride_c = M * N if stride_c is None else stride_c
     if out is None:
         out = torch.empty(max(batch * stride_c, 1), dtype=torch.bfloat16, device=DEV)
-    fp8.fp8_mm(a8, fa, b8, fb, sa, sb, layout, M, N, K, batch, stride_a, stride_b, stride_c,
-               bias, bias_scale, bias_fmt, out)
+    if ws is None and split_k == 0:
+        fp8.fp8_mm(a8, fa, b8, fb, sa, sb, layout, M, N, K, batch, stride_a, stride_b, stride_c,
+                   bias, bias_scale, bias_fmt, out)
+    else:
+        fp8.fp8_mm_ws(a8, fa, b8, fb, sa, sb, layout, M, N, K, batch, stride_a, stride_b, stride_c,
+                      bias, bias_scale, bias_fmt, out, ws, split_k)
     return out
+
+
+def workspace(nbytes):
+    """A zero-filled GEMM workspace (uint8)."""
+    return torch.zeros(max(int(nbytes), 4096), dtype=torch.uint8, device=DEV)
 
 
 def assert_within(got, want, tol, what=""):

@@ -123,3 +123,28 @@ def test_quantize_many_validation(fp8):
     assert status([(A, 64, 5, S, A + 4096, None, S + 64)]) == fp8.FP8_ERR_INVALID_ARG     # bad fmt
     assert status([(A + 2, 64, 0, S, A + 4096, None, S + 64)]) == fp8.FP8_ERR_ALIGNMENT
     assert fp8.raw_status("fp8_quantize_many", None, 1, None) == fp8.FP8_ERR_INVALID_ARG
+
+
+def test_mm_workspace_size_and_alignment(fp8):
+    # no split requested or chosen: no workspace
+    assert fp8.fp8_mm_workspace_size(2048, 1024, 4096, 1, fp8.FP8_NT, 0) == 0
+    assert fp8.fp8_mm_workspace_size(2048, 1024, 4096, 1, fp8.FP8_NT, 1) == 0
+    # two splits: the counters plus at least two fp32 partials of the whole output
+    assert fp8.fp8_mm_workspace_size(2048, 1024, 4096, 1, fp8.FP8_NT, 2) >= 4096 + 2 * 2048 * 1024 * 4
+    assert fp8.fp8_mm_workspace_size(1, 4096, 4096, 1, fp8.FP8_NT, 4) >= 4096 + 4 * 128 * 4096 * 4
+    # too many tile halves for the counters, too few k-blocks, bad arguments
+    assert fp8.fp8_mm_workspace_size(8192, 8192, 8192, 1, fp8.FP8_NT, 2) == 0
+    assert fp8.fp8_mm_workspace_size(2048, 1024, 256, 1, fp8.FP8_NT, 4) == 0
+    assert fp8.fp8_mm_workspace_size(0, 8, 8, 1, fp8.FP8_NT, 2) == 0
+    assert fp8.fp8_mm_workspace_size(8, 8, 8, 1, 7, 2) == 0
+    assert fp8.fp8_mm_workspace_size(8, 8, 1024, 1, fp8.FP8_NT, 5) == 0
+    st = fp8.raw_status("fp8_mm_ws", A, 0, A, 0, S, S, 0, 16, 16, 16, 1, 256, 256, 256, None, None, 0, A,
+                        A + 8, 1 << 20, 2, None)
+    assert st == fp8.FP8_ERR_ALIGNMENT
+    st = fp8.raw_status("fp8_mm_ws", A, 0, A, 0, S, S, 9, 16, 16, 16, 1, 256, 256, 256, None, None, 0, A,
+                        A, 1 << 20, 2, None)
+    assert st == fp8.FP8_ERR_INVALID_ARG
+    for split_k in (-1, 5):
+        st = fp8.raw_status("fp8_mm_ws", A, 0, A, 0, S, S, 0, 16, 16, 16, 1, 256, 256, 256, None, None, 0, A,
+                            A, 1 << 20, split_k, None)
+        assert st == fp8.FP8_ERR_INVALID_ARG

@@ -211,3 +211,16 @@ def test_pair_tiles_full(g, layout, M, N, K):
 def test_pair_tiles_bias_and_batches(g, layout):
     _full_check(g, layout, 1280, 2560, 256, E5M2, E4M3, 1101, batch=3, bcast_b=True, pad_c=48, bias_kind=1)
     _full_check(g, layout, 2560, 4096, 128, E4M3, E5M2, 1102, bias_kind=2)
+
+
+# Narrow NT problems with a long K (few output tiles, many k-blocks): ragged
+# M and N, bias of both kinds, broadcast batches.
+
+@pytest.mark.parametrize("M,N,K,bias_kind", [(512, 512, 2048, 0), (1000, 1000, 1024, 1), (2048, 1024, 1024, 2),
+                                             (136, 200, 4096, 1), (2048, 1024, 4096, 0)])
+def test_narrow_long_k_nt(g, M, N, K, bias_kind):
+    _full_check(g, NT, M, N, K, E4M3, E4M3, 1200 + M + N, bias_kind=bias_kind)
+
+
+def test_narrow_long_k_nt_batches(g):
+    _full_check(g, NT, 384, 640, 1024, E4M3, E5M2, 1301, batch=2, bcast_b=True, pad_c=32, bias_kind=1)
