@@ -71,6 +71,8 @@ def _load():
         "fp8_mm_ws": (I, [P, I, P, I, P, P, I, I64, I64, I64, I64, I64, I64, I64, P, P, I, P, P, ctypes.c_size_t,
                           ctypes.c_int32, P]),
         "fp8_mm_workspace_size": (ctypes.c_size_t, [I64, I64, I64, I64, I, ctypes.c_int32]),
+        "fp8_mm_splitk_static": (I, [P, I, P, I, P, P, I, I64, I64, I64, I64, I64, I64, I64, P, P, I, P,
+                                     ctypes.c_int32, P]),
     }
     for name, (res, args) in sig.items():
         try:
@@ -168,6 +170,15 @@ def fp8_mm_ws(a8, fa, b8, fb, sa, sb, layout, M, N, K, batch, stride_a, stride_b
 
 def fp8_mm_workspace_size(M, N, K, batch, layout, split_k):
     return int(lib.fp8_mm_workspace_size(int(M), int(N), int(K), int(batch), int(layout), int(split_k)))
+
+
+def fp8_mm_splitk_static(a8, fa, b8, fb, sa, sb, layout, M, N, K, batch, stride_a, stride_b, stride_c, bias,
+                         bias_scale, bias_fmt, out, split_k, stream=None):
+    """Split-K fp8_mm on the library's own scratch (no workspace argument)."""
+    return _check(lib.fp8_mm_splitk_static(_ptr(a8), int(fa), _ptr(b8), int(fb), _ptr(sa), _ptr(sb), int(layout),
+                                           int(M), int(N), int(K), int(batch), int(stride_a), int(stride_b),
+                                           int(stride_c), _ptr(bias), _ptr(bias_scale), int(bias_fmt), _ptr(out),
+                                           int(split_k), _stream(stream)), "fp8_mm_splitk_static")
 
 
 def fp8_last_device_error():

@@ -874,6 +874,28 @@ extern "C" size_t fp8_mm_workspace_size(int64_t M, int64_t N, int64_t K, int64_t
     return split_ws_bytes(tile_count(M, N, batch, tc.pair, tc.bn), tc.pair ? 2 : 1, tc.bn, tc.split);
 }
 
+// Library-owned split-K scratch for fp8_mm_splitk_static: the counters (zero
+// from module load, left zero by every completed call) and the fp32 partial
+// tiles, so that a split GEMM needs no allocation from the caller or the
+// library.
+constexpr size_t kStaticScratchBytes = size_t(32) << 20;
+__device__ __align__(256) uint8_t g_splitk_scratch[kStaticScratchBytes];
+
+extern "C" fp8_status fp8_mm_splitk_static(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8, fp8_fmt fb,
+                                           const float* sa, const float* sb, fp8_layout layout, int64_t M, int64_t N,
+                                           int64_t K, int64_t batch, int64_t stride_a, int64_t stride_b,
+                                           int64_t stride_c, const void* bias, const float* bias_scale,
+                                           fp8_fmt bias_fmt, void* out, int32_t split_k, void* stream) {
+    if (split_k < 2 || split_k > kMaxSplit) return FP8_ERR_INVALID_ARG;
+    const size_t need = fp8_mm_workspace_size(M, N, K, batch, layout, split_k);
+    if (need > kStaticScratchBytes) return FP8_ERR_UNSUPPORTED;
+    void* scratch = nullptr;
+    if (cudaGetSymbolAddress(&scratch, g_splitk_scratch) != cudaSuccess) return FP8_ERR_CUDA;
+    // fp8_mm_ws validates the rest (and reports a split the problem cannot take)
+    return fp8_mm_ws(a8, fa, b8, fb, sa, sb, layout, M, N, K, batch, stride_a, stride_b, stride_c, bias, bias_scale,
+                     bias_fmt, out, scratch, kStaticScratchBytes, split_k, stream);
+}
+
 extern "C" fp8_status fp8_last_device_error(void) {
     if (cudaDeviceSynchronize() != cudaSuccess) return FP8_ERR_CUDA;
     uint32_t v = 0;

@@ -231,6 +231,22 @@ FP8LITE_API fp8_status fp8_mm_ws(const uint8_t* a8, fp8_fmt fa, const uint8_t* b
 FP8LITE_API size_t fp8_mm_workspace_size(int64_t M, int64_t N, int64_t K, int64_t batch, fp8_layout layout,
                                          int32_t split_k);
 
+/* fp8_mm_ws with split_k = 2 .. 4 on scratch the library owns: a 32 MiB
+ * device array of the library (zero from load, its counters left zero by
+ * every completed call), so the call allocates nothing and needs no
+ * workspace from the caller. Same result, bit for bit, as fp8_mm_ws with the
+ * same split_k. The scratch is one per device: calls that may run at the same
+ * time on one device (e.g. on two streams) must not use this entry point.
+ * Errors: as fp8_mm_ws; FP8_ERR_INVALID_ARG for split_k outside 2 .. 4;
+ * FP8_ERR_UNSUPPORTED when the split needs more than the 32 MiB
+ * (fp8_mm_workspace_size() > 33554432) or the problem cannot take it. */
+FP8LITE_API fp8_status fp8_mm_splitk_static(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8, fp8_fmt fb,
+                  const float* sa, const float* sb, fp8_layout layout,
+                  int64_t M, int64_t N, int64_t K, int64_t batch,
+                  int64_t stride_a, int64_t stride_b, int64_t stride_c,
+                  const void* bias, const float* bias_scale, fp8_fmt bias_fmt,
+                  void* out, int32_t split_k, void* stream);
+
 /* Synchronises the current device, then reads and clears the library's
  * device error word: FP8_ERR_DEVICE_TIMEOUT if a GEMM thread block gave up a
  * bounded wait since the last call (its output tile is then undefined),
