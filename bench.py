@@ -736,6 +736,19 @@ def run_kernel(args):
         call = lambda i: fp8.fp8_mm_ws(sets[i % 2][0], E4M3, sets[i % 2][1], E4M3, sa, sa, layout, M, N, K, 1, 0, 0,
                                        0, None, None, 0, out, ws, args.split_k if need else 0, stream=st)
         units = 2.0 * M * N * K
+    elif args.kernel == "quantize_many":
+        # the linear stack's step-start launch: every weight and the first x
+        sizes = [d_out * d_in for _, d_in, d_out in W.LINEARS] + [W.TOKENS * W.LINEARS[0][1]]
+        xs = [[W.bf16_normal((n,), 1.0, 9400 + 10 * i + j).cuda() for j, n in enumerate(sizes)] for i in range(2)]
+        qs = [torch.empty(n, dtype=torch.uint8, device="cuda") for n in sizes]
+        rings = [torch.empty(20, dtype=torch.int32, device="cuda") for _ in sizes]
+        for r in rings:
+            fp8.fp8_ring_init(r, 1.0)
+        scs = [torch.empty(1, device="cuda") for _ in sizes]
+        ams = [torch.empty(1, device="cuda") for _ in sizes]
+        jobs = [[(xs[i][j], n, E4M3, rings[j], qs[j], ams[j], scs[j]) for j, n in enumerate(sizes)] for i in range(2)]
+        call = lambda i: fp8.fp8_quantize_many(jobs[i % 2], stream=st)
+        units = 3.0 * sum(sizes)
     else:
         n = int(args.shape)
         xs = [W.bf16_normal((n,), 1.0, 9300 + i).cuda() for i in range(2)]
@@ -768,7 +781,7 @@ def run_kernel(args):
                           "peak_source": src}))
     else:
         ach = units / (us * 1e-6) / 1e9
-        print(json.dumps({"kernel": "quantize", "n": int(args.shape), "us": round(us, 2), "gbs": round(ach, 1),
+        print(json.dumps({"kernel": args.kernel, "n": int(units / 3), "us": round(us, 2), "gbs": round(ach, 1),
                           "frac_hbm": round(ach / hbm, 4), "peak": hbm, "peak_source": src}))
 
 
@@ -787,7 +800,7 @@ def main():
     ap.add_argument("--no-compare", action="store_true", help="skip the bf16 / autograd comparison")
     ap.add_argument("--breakdown-reps", type=int, default=20)
     ap.add_argument("--e2e-steps", type=int, default=10)
-    ap.add_argument("--kernel", choices=["gemm", "quantize", "cublaslt"], help="single-kernel mode")
+    ap.add_argument("--kernel", choices=["gemm", "quantize", "quantize_many", "cublaslt"], help="single-kernel mode")
     ap.add_argument("--shape", default="8192x8192x8192", help="MxNxK for gemm, n for quantize")
     ap.add_argument("--layout", default="NT", choices=["NT", "NN", "TN"])
     args = ap.parse_args()
