@@ -104,6 +104,21 @@ __device__ __forceinline__ void quantize_body(const uint16_t* __restrict__ x, in
                                               fp8_ring* ring, uint32_t* amax_acc, float* amax_out, float* scale_out,
                                               int blk, int nblk, float& s_scale) {
     const float fmax = fmt_max(FMT);
+    const uint4* xv = reinterpret_cast<const uint4*>(x);
+    uint2* ov = reinterpret_cast<uint2*>(out8);
+    const int64_t units = n >> 3;  // 8 elements per unit
+    const int64_t tid = int64_t(blk) * kThreads + threadIdx.x;
+    const int64_t stride = int64_t(nblk) * kThreads;
+    // The first round of input loads leaves before the scale is known (the
+    // loads do not need it); for tensors of up to 2048 elements per thread
+    // of the grid that is every load.
+    int64_t base = tid;
+    uint4 v[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const int64_t i = base + u * stride;
+        if (i < units) v[u] = __ldg(xv + i);
+    }
     // One thread per block reads the scale (or the amax it comes from) and
     // shares it: thousands of warps loading one address would queue on a
     // single L2 line.
@@ -122,21 +137,9 @@ __device__ __forceinline__ void quantize_body(const uint16_t* __restrict__ x, in
         __syncthreads();
     }
     const float s = MODE == kAmaxOnly ? 1.0f : s_scale;
-
-    const uint4* xv = reinterpret_cast<const uint4*>(x);
-    uint2* ov = reinterpret_cast<uint2*>(out8);
-    const int64_t units = n >> 3;  // 8 elements per unit
-    const int64_t tid = int64_t(blk) * kThreads + threadIdx.x;
-    const int64_t stride = int64_t(nblk) * kThreads;
     float m = 0.0f;
 
-    for (int64_t base = tid; base < units; base += stride * kUnroll) {
-        uint4 v[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int64_t i = base + u * stride;
-            if (i < units) v[u] = __ldg(xv + i);
-        }
+    while (base < units) {
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
             const int64_t i = base + u * stride;
@@ -151,6 +154,13 @@ __device__ __forceinline__ void quantize_body(const uint16_t* __restrict__ x, in
                     ov[i] = q;
                 }
             }
+        }
+        base += stride * kUnroll;
+        if (base >= units) break;
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t i = base + u * stride;
+            if (i < units) v[u] = __ldg(xv + i);
         }
     }
     griddep_launch();  // the next kernel may start its prologue
@@ -174,18 +184,20 @@ __device__ __forceinline__ void quantize_body(const uint16_t* __restrict__ x, in
     // ticket moves); the block holding the final ticket sees every amax.
     const uint32_t ticket = atom_add_acq_rel(&ring->ticket, 1u);
     if (ticket != uint32_t(nblk) - 1) return;
-    const float a = __uint_as_float(atomicExch(&ring->amax_bits, 0u));
+    // The history and its index change only in this finalize, so they are
+    // read together with the exchange of the accumulated amax: the 18
+    // accesses leave at once and cost one round trip to L2.
     volatile fp8_ring* r = ring;
-    // the window's maximum over the 15 kept entries and the new amax; the
-    // loop is unrolled so the 17 independent loads leave together (a rolled
-    // loop serialises them into 17 round trips to L2)
+    float h[FP8_RING_HISTORY];
+#pragma unroll
+    for (int i = 0; i < FP8_RING_HISTORY; ++i) h[i] = r->hist[i];
     const uint32_t idx = r->idx & (FP8_RING_HISTORY - 1);
+    const float a = __uint_as_float(atomicExch(&ring->amax_bits, 0u));
+    // the window's maximum over the 15 kept entries and the new amax
     float wmax = a;
 #pragma unroll
-    for (int i = 0; i < FP8_RING_HISTORY; ++i) {
-        const float v = r->hist[i];
-        if (uint32_t(i) != idx) wmax = fmaxf(wmax, v);
-    }
+    for (int i = 0; i < FP8_RING_HISTORY; ++i)
+        if (uint32_t(i) != idx) wmax = fmaxf(wmax, h[i]);
     r->hist[idx] = a;
     if (wmax > 0.0f && isfinite(wmax)) r->scale = scale_from_amax(fmax, wmax);
     r->idx = (idx + 1) & (FP8_RING_HISTORY - 1);
