@@ -230,7 +230,7 @@ __device__ __forceinline__ bool epilogue_bar_or(bool v) {
 // Epilogue: 4 warps, one per TMEM lane quarter. Every 32 columns of the tile
 // become a 128 x 32 bf16 tile in shared memory that one thread writes with a
 // single TMA store (8 stores for a 128 x 256 tile).
-template <int BN, bool A_MN, bool B_MN, int STAGES, bool HAS_BIAS, int CTAS, bool SPLIT>
+template <int BN, bool A_MN, bool B_MN, int STAGES, bool HAS_BIAS, int CTAS, bool SPLIT, bool SWAP>
 __global__ void __maxnreg__(168)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const __grid_constant__ CUtensorMap tm_c, const GemmParams p) {
@@ -403,7 +403,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             const int buf = it & 1;
             const uint32_t acc_phase = (it >> 1) & 1;
             const int m0 = mb * BM * CTAS + int(rank) * BM;  // this CTA's first output row
-            if (HAS_BIAS) {
+            if (HAS_BIAS && !SWAP) {
                 // the tile's BN bias values, dequantized once into shared memory
                 epilogue_bar();  // the previous tile's readers are done
                 for (int j = etid; j < BN; j += kEpiThreads) {
@@ -432,9 +432,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             const uint32_t t_row = tmem_base + (uint32_t(q * 32) << 16) + buf * BN;
             // Split K: the unit that arrives last at its tile finishes it; the
             // others leave their fp32 partial in the workspace. Slot layout:
-            // 16-byte piece v of 32-column chunk c of tile row r sits at
-            // ((c * 8 + v) * 128 + r) * 16, so each store and load instruction
-            // of a warp covers 512 contiguous bytes.
+            // 16-byte piece v of CW-column chunk c of tile row r sits at
+            // ((c * CW / 4 + v) * 128 + r) * 16, so each store and load
+            // instruction of a warp covers 512 contiguous bytes.
+            constexpr int CW = SWAP ? 16 : 32;  // accumulator columns per TMEM load
             const float4* slots = nullptr;
             if (SPLIT && split > 1) {
                 uint32_t* cnt = p.ws_cnt + 2 * (t * CTAS + int(rank));
@@ -445,14 +446,14 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                 if (!last) {
                     float4* mine = const_cast<float4*>(slots) + size_t(split_id) * (BM * BN / 4);
 #pragma unroll 1
-                    for (int c = 0; c < BN / 32; ++c) {
-                        if (nb * BN + c * 32 >= N) break;  // uniform; the finisher skips it too
-                        uint32_t r[32];
-                        tmem_ld32(t_row + c * 32, r);
+                    for (int c = 0; c < BN / CW; ++c) {
+                        if (nb * BN + c * CW >= N) break;  // uniform; the finisher skips it too
+                        uint32_t r[CW];
+                        tmem_ld<CW>(t_row + c * CW, r);
                         tmem_ld_wait();
 #pragma unroll
-                        for (int v = 0; v < 8; ++v)
-                            __stcg(mine + (c * 8 + v) * 128 + row_in_tile,
+                        for (int v = 0; v < CW / 4; ++v)
+                            __stcg(mine + (c * (CW / 4) + v) * 128 + row_in_tile,
                                    make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
                                                __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])));
                     }
@@ -472,28 +473,40 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                 epilogue_bar();
             }
             const int row = m0 + row_in_tile;
-            uint16_t* orow = p.out + int64_t(b) * p.stride_c + int64_t(row) * N;
+            // swapped operands: this thread's TMEM lane is output column `row`
+            // of C (the kernel's M is C's N), its accumulator columns are C's rows
+            float bias_row = 0.0f;
+            if (SWAP && HAS_BIAS && row < M) {
+                if (p.bias_kind == 1)
+                    bias_row = __uint_as_float(uint32_t(__ldg(static_cast<const uint16_t*>(p.bias) + row)) << 16);
+                else
+                    bias_row = __fdiv_rn(fp8_to_f32(__ldg(static_cast<const uint8_t*>(p.bias) + row), p.bias_fmt),
+                                         bscale);
+            }
+            uint16_t* orow = SWAP ? p.out + int64_t(b) * p.stride_c + row
+                                  : p.out + int64_t(b) * p.stride_c + int64_t(row) * N;
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                const int col0 = nb * BN + c * 32;
+            for (int c = 0; c < BN / CW; ++c) {
+                const int col0 = nb * BN + c * CW;
                 if (col0 >= N) break;  // uniform over the epilogue warps
-                uint32_t r[32];
-                tmem_ld32(t_row + c * 32, r);
+                uint32_t r[CW];
+                tmem_ld<CW>(t_row + c * CW, r);
                 tmem_ld_wait();
                 if (SPLIT && split > 1) {
                     // the sum over the splits in split order, whatever order
                     // they arrived in (the result does not depend on timing)
-                    float acc[32];
+                    float acc[CW];
 #pragma unroll 1
                     for (int sp = 0; sp < split; ++sp) {
                         if (sp == split_id) {
 #pragma unroll
-                            for (int i = 0; i < 32; ++i)
+                            for (int i = 0; i < CW; ++i)
                                 acc[i] = sp == 0 ? __uint_as_float(r[i]) : acc[i] + __uint_as_float(r[i]);
                         } else {
-                            const float4* src = slots + size_t(sp) * (BM * BN / 4) + c * 8 * 128 + row_in_tile;
+                            const float4* src =
+                                slots + size_t(sp) * (BM * BN / 4) + c * (CW / 4) * 128 + row_in_tile;
 #pragma unroll
-                            for (int v = 0; v < 8; ++v) {
+                            for (int v = 0; v < CW / 4; ++v) {
                                 const float4 x = __ldcg(src + v * 128);
                                 acc[4 * v] = sp == 0 ? x.x : acc[4 * v] + x.x;
                                 acc[4 * v + 1] = sp == 0 ? x.y : acc[4 * v + 1] + x.y;
@@ -503,59 +516,74 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                         }
                     }
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(acc[i]);
+                    for (int i = 0; i < CW; ++i) r[i] = __float_as_uint(acc[i]);
                 }
-                float y[32];
+                if constexpr (SWAP) {
+                    // C[col0 + i][row]: lanes hold consecutive columns, so each
+                    // store instruction of a warp writes 64 contiguous bytes
+                    if (row < M) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float bias = HAS_BIAS ? s_bias[c * 32 + i] : 0.0f;
-                    y[i] = fmaf(__uint_as_float(r[i]), inv, bias);
-                }
-                if (tma_store) {
-                    // the 128 x 32 bf16 block goes to the staging tile whose last
-                    // store is known to have read it (64-byte swizzle: 16-byte
-                    // piece j of row r at (j ^ (r / 2 mod 4)) * 16, so the 8
-                    // lanes of a store phase hit distinct banks); then one TMA
-                    // store, which clips the M / N tails of the output
-                    const uint32_t stg = stg0 + (n_st & 1) * L::kStgBytes;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const uint32_t addr = stg + row_in_tile * 64 + ((j ^ ((row_in_tile >> 1) & 3)) << 4);
-                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
-                                     "r"(pack_bf16x2(y[8 * j + 0], y[8 * j + 1])),
-                                     "r"(pack_bf16x2(y[8 * j + 2], y[8 * j + 3])),
-                                     "r"(pack_bf16x2(y[8 * j + 4], y[8 * j + 5])),
-                                     "r"(pack_bf16x2(y[8 * j + 6], y[8 * j + 7]))
-                                     : "memory");
-                    }
-                    fence_proxy_async_smem();
-                    // the previous store has read the other tile, which the next
-                    // block reuses; the barrier publishes that and this block
-                    if (store_lead) bulk_wait_read<0>();
-                    epilogue_bar();
-                    if (store_lead) {
-                        tma_store_3d(&tm_c, stg, col0, m0, b);
-                        bulk_commit();
-                    }
-                    ++n_st;
-                } else if (row < M) {
-                    if (vec_store && col0 + 32 <= N) {
-                        uint4* dst = reinterpret_cast<uint4*>(orow + col0);
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            uint4 x;
-                            x.x = pack_bf16x2(y[8 * v + 0], y[8 * v + 1]);
-                            x.y = pack_bf16x2(y[8 * v + 2], y[8 * v + 3]);
-                            x.z = pack_bf16x2(y[8 * v + 4], y[8 * v + 5]);
-                            x.w = pack_bf16x2(y[8 * v + 6], y[8 * v + 7]);
-                            dst[v] = x;
+                        for (int i = 0; i < CW; ++i) {
+                            if (col0 + i >= N) break;
+                            const float y = fmaf(__uint_as_float(r[i]), inv, bias_row);
+                            uint16_t h;
+                            asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(h) : "f"(y));
+                            orow[int64_t(col0 + i) * M] = h;
                         }
-                    } else {
+                    }
+                } else {
+                    float y[CW];
 #pragma unroll
-                        for (int i = 0; i < 32; i += 2) {
-                            const uint32_t x = pack_bf16x2(y[i], y[i + 1]);
-                            if (col0 + i < N) orow[col0 + i] = uint16_t(x & 0xFFFFu);
-                            if (col0 + i + 1 < N) orow[col0 + i + 1] = uint16_t(x >> 16);
+                    for (int i = 0; i < CW; ++i) {
+                        const float bias = HAS_BIAS ? s_bias[c * CW + i] : 0.0f;
+                        y[i] = fmaf(__uint_as_float(r[i]), inv, bias);
+                    }
+                    if (tma_store) {
+                        // the 128 x 32 bf16 block goes to the staging tile whose last
+                        // store is known to have read it (64-byte swizzle: 16-byte
+                        // piece j of row r at (j ^ (r / 2 mod 4)) * 16, so the 8
+                        // lanes of a store phase hit distinct banks); then one TMA
+                        // store, which clips the M / N tails of the output
+                        const uint32_t stg = stg0 + (n_st & 1) * L::kStgBytes;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const uint32_t addr = stg + row_in_tile * 64 + ((j ^ ((row_in_tile >> 1) & 3)) << 4);
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                                         "r"(pack_bf16x2(y[8 * j + 0], y[8 * j + 1])),
+                                         "r"(pack_bf16x2(y[8 * j + 2], y[8 * j + 3])),
+                                         "r"(pack_bf16x2(y[8 * j + 4], y[8 * j + 5])),
+                                         "r"(pack_bf16x2(y[8 * j + 6], y[8 * j + 7]))
+                                         : "memory");
+                        }
+                        fence_proxy_async_smem();
+                        // the previous store has read the other tile, which the next
+                        // block reuses; the barrier publishes that and this block
+                        if (store_lead) bulk_wait_read<0>();
+                        epilogue_bar();
+                        if (store_lead) {
+                            tma_store_3d(&tm_c, stg, col0, m0, b);
+                            bulk_commit();
+                        }
+                        ++n_st;
+                    } else if (row < M) {
+                        if (vec_store && col0 + 32 <= N) {
+                            uint4* dst = reinterpret_cast<uint4*>(orow + col0);
+#pragma unroll
+                            for (int v = 0; v < 4; ++v) {
+                                uint4 x;
+                                x.x = pack_bf16x2(y[8 * v + 0], y[8 * v + 1]);
+                                x.y = pack_bf16x2(y[8 * v + 2], y[8 * v + 3]);
+                                x.z = pack_bf16x2(y[8 * v + 4], y[8 * v + 5]);
+                                x.w = pack_bf16x2(y[8 * v + 6], y[8 * v + 7]);
+                                dst[v] = x;
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; i += 2) {
+                                const uint32_t x = pack_bf16x2(y[i], y[i + 1]);
+                                if (col0 + i < N) orow[col0 + i] = uint16_t(x & 0xFFFFu);
+                                if (col0 + i + 1 < N) orow[col0 + i + 1] = uint16_t(x >> 16);
+                            }
                         }
                     }
                 }
@@ -657,11 +685,11 @@ struct HostArgs {
     int64_t batch, stride_b;
 };
 
-template <int BN, bool A_MN, bool B_MN, int STAGES, bool HAS_BIAS, int CTAS, bool SPLIT>
+template <int BN, bool A_MN, bool B_MN, int STAGES, bool HAS_BIAS, int CTAS, bool SPLIT, bool SWAP>
 fp8_status launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, GemmParams p,
                       const HostArgs& h, cudaStream_t st) {
     using L = Smem<BN, STAGES, CTAS>;
-    auto kern = fp8_gemm_kernel<BN, A_MN, B_MN, STAGES, HAS_BIAS, CTAS, SPLIT>;
+    auto kern = fp8_gemm_kernel<BN, A_MN, B_MN, STAGES, HAS_BIAS, CTAS, SPLIT, SWAP>;
     static bool attr_set[64] = {false};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8_ERR_CUDA;
@@ -684,15 +712,15 @@ fp8_status launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
     return launch_pdl(kern, units * CTAS, kThreads, L::kAlloc, st, CTAS, ta, tb, tc, p);
 }
 
-template <int BN, bool A_MN, bool B_MN, int STAGES, int CTAS>
+template <int BN, bool A_MN, bool B_MN, int STAGES, int CTAS, bool SWAP = false>
 fp8_status launch(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, const HostArgs& h, cudaStream_t st) {
     CUtensorMap tc = {};
     if (p.tma_store && !make_out_map(&tc, p.out, p.N, p.M, h.batch, uint64_t(p.stride_c) * 2)) return FP8_ERR_CUDA;
     if (p.split > 1)
-        return p.bias_kind ? launch_one<BN, A_MN, B_MN, STAGES, true, CTAS, true>(ta, tb, tc, p, h, st)
-                           : launch_one<BN, A_MN, B_MN, STAGES, false, CTAS, true>(ta, tb, tc, p, h, st);
-    return p.bias_kind ? launch_one<BN, A_MN, B_MN, STAGES, true, CTAS, false>(ta, tb, tc, p, h, st)
-                       : launch_one<BN, A_MN, B_MN, STAGES, false, CTAS, false>(ta, tb, tc, p, h, st);
+        return p.bias_kind ? launch_one<BN, A_MN, B_MN, STAGES, true, CTAS, true, SWAP>(ta, tb, tc, p, h, st)
+                           : launch_one<BN, A_MN, B_MN, STAGES, false, CTAS, true, SWAP>(ta, tb, tc, p, h, st);
+    return p.bias_kind ? launch_one<BN, A_MN, B_MN, STAGES, true, CTAS, false, SWAP>(ta, tb, tc, p, h, st)
+                       : launch_one<BN, A_MN, B_MN, STAGES, false, CTAS, false, SWAP>(ta, tb, tc, p, h, st);
 }
 
 // Tile choice for 148 SMs by a small cost model: a persistent grid walks
@@ -785,6 +813,81 @@ fp8_status dispatch(const CUtensorMap& ta, GemmParams p, const HostArgs& h, void
     return FP8_ERR_UNSUPPORTED;
 }
 
+// Swapped operands for short problems (M <= 32, N >= 128, NT or NN): the
+// kernel computes C^T = B^T A^T, so that C's N runs along the tensor core's
+// 128-row M and C's few rows become an MMA N of 16 or 32; the epilogue
+// writes C transposed. (TN is excluded: its A would become an MN-major B
+// operand narrower than a 128-byte swizzle atom. From 33 rows on, the
+// unswapped 128 x 64 tile was as fast or faster on B200: at 64 x 8192 x 2048
+// it keeps 128 SMs busy where the swapped 128 x 64 tiles keep 64.)
+inline bool swap_ab(int64_t M, int64_t N, fp8_layout layout) {
+    return M <= 32 && N >= 128 && layout != FP8_TN;
+}
+
+inline int swap_bn(int64_t M) { return M <= 16 ? 16 : 32; }
+
+// The split a swapped problem takes (0: the requested split is impossible).
+// Automatic (split_req 0): few 128-column tiles with a long K leave most SMs
+// idle, and their partials are small (128 x 16..64 fp32), so splitting pays
+// where the main loop it saves exceeds the fix-up: about 0.28 us per k-block
+// saved against 2.2 + 0.02 * BN * split us, with every unit in one round (both
+// constants measured on B200 over 1, 8, 16, 32 and 64-row problems).
+inline int swap_split(int64_t M, int64_t N, int64_t K, int64_t batch, int split_req, int64_t sms) {
+    const int64_t kb = (K + BK - 1) / BK;
+    const int64_t tiles = ((N + BM - 1) / BM) * batch;
+    auto possible = [&](int s) {
+        const int64_t kb_per = (kb + s - 1) / s;
+        return (s - 1) * kb_per < kb && size_t(tiles) * 2 * sizeof(uint32_t) <= kSplitCntBytes;
+    };
+    if (split_req == 1) return 1;
+    if (split_req >= 2) return possible(split_req) ? split_req : 0;
+    const int bn = swap_bn(M);
+    int best = 1;
+    double best_gain = 0.0;
+    for (int s = 2; s <= kMaxSplit; ++s) {
+        if (!possible(s) || tiles * s > sms) continue;
+        const double gain = double(kb - (kb + s - 1) / s) * 0.28 - (2.2 + 0.02 * bn * s);
+        if (gain > best_gain) { best = s; best_gain = gain; }
+    }
+    return best;
+}
+
+template <bool A_MN>
+fp8_status dispatch_swap(const uint8_t* a8, int fa, const uint8_t* b8, int fb, int64_t M, int64_t N, int64_t K,
+                         int64_t batch, int64_t stride_a, int64_t stride_b, GemmParams p, void* ws, size_t ws_bytes,
+                         int split_req, cudaStream_t st) {
+    const int bn = swap_bn(M);
+    // the automatic choice splits only with a workspace to split into
+    p.split = swap_split(M, N, K, batch, split_req == 0 && !ws ? 1 : split_req, sm_count());
+    if (p.split == 0) return FP8_ERR_UNSUPPORTED;
+    if (p.split > 1) {
+        const int64_t tiles = ((N + BM - 1) / BM) * batch;
+        if (!ws || ws_bytes < split_ws_bytes(tiles, 1, bn, p.split)) {
+            if (split_req >= 2) return FP8_ERR_INVALID_ARG;
+            p.split = 1;  // an automatic split that does not fit the workspace is dropped
+        }
+    }
+    if (p.split > 1) {
+        p.ws_cnt = static_cast<uint32_t*>(ws);
+        p.ws = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kSplitCntBytes);
+    }
+    // the kernel's problem: M' = N rows of A' = B, N' = M columns of B' = A
+    p.M = int(N);
+    p.N = int(M);
+    p.a_bcast = stride_b == 0;
+    p.b_bcast = stride_a == 0;
+    p.tma_store = 0;
+    p.vec_store = 0;
+    CUtensorMap ta, tb;
+    const bool ok_a = A_MN ? make_map(&ta, b8, N, K, batch, uint64_t(stride_b), 128, BK)
+                           : make_map(&ta, b8, K, N, batch, uint64_t(stride_b), BK, BM);
+    const bool ok_b = make_map(&tb, a8, K, M, batch, uint64_t(stride_a), BK, uint32_t(bn));
+    if (!ok_a || !ok_b) return FP8_ERR_CUDA;
+    const HostArgs h = {fb, fa, a8, batch, stride_a};
+    if (bn == 16) return launch<16, A_MN, false, 10, 1, true>(ta, tb, p, h, st);
+    return launch<32, A_MN, false, 9, 1, true>(ta, tb, p, h, st);
+}
+
 }  // namespace
 }  // namespace fp8lite
 
@@ -841,12 +944,17 @@ extern "C" fp8_status fp8_mm_ws(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8
     p.split = 1;
     p.vec_store = (N % 8 == 0) && (stride_c % 8 == 0) && aligned(out, 16);
     p.tma_store = p.vec_store;
+    cudaStream_t st = as_stream(stream);
+    if (swap_ab(M, N, layout))
+        return layout == FP8_NN ? dispatch_swap<true>(a8, fa, b8, fb, M, N, K, batch, stride_a, stride_b, p, workspace,
+                                                      workspace_bytes, split_k, st)
+                                : dispatch_swap<false>(a8, fa, b8, fb, M, N, K, batch, stride_a, stride_b, p,
+                                                       workspace, workspace_bytes, split_k, st);
 
     CUtensorMap ta;
     bool ok = a_mn ? make_map(&ta, a8, M, K, batch, uint64_t(stride_a), 128, BK)
                    : make_map(&ta, a8, K, M, batch, uint64_t(stride_a), BK, BM);
     if (!ok) return FP8_ERR_CUDA;
-    cudaStream_t st = as_stream(stream);
     const HostArgs h = {int(fa), int(fb), b8, batch, stride_b};
     switch (layout) {
         case FP8_NT: return dispatch<false, false>(ta, p, h, workspace, workspace_bytes, split_k, st);
@@ -869,6 +977,11 @@ extern "C" size_t fp8_mm_workspace_size(int64_t M, int64_t N, int64_t K, int64_t
     if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31) || batch >= (int64_t(1) << 31))
         return 0;
     if (layout != FP8_NT && layout != FP8_NN && layout != FP8_TN) return 0;
+    if (swap_ab(M, N, layout)) {
+        const int split = swap_split(M, N, K, batch, split_k, sm_count());
+        if (split < 2) return 0;
+        return split_ws_bytes(((N + BM - 1) / BM) * batch, 1, swap_bn(M), split);
+    }
     const TileChoice tc = choose_tile(M, N, K, batch, layout != FP8_NT, sm_count(), split_k);
     if (tc.split < 2) return 0;
     return split_ws_bytes(tile_count(M, N, batch, tc.pair, tc.bn), tc.pair ? 2 : 1, tc.bn, tc.split);

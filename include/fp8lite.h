@@ -197,11 +197,17 @@ FP8LITE_API fp8_status fp8_mm(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8, 
  * and it is deterministic: it does not depend on the order in which the
  * splits finish.
  *
- * split_k         0: the library's choice (in this version: no split -- on
- *                 every shape measured on B200 the partials' round trip
- *                 through L2 cost more than the shorter main loop saved);
+ * split_k         0: the library's choice: it splits only short problems
+ *                 (M <= 32, NT or NN; they run with swapped operands, so a
+ *                 tile is 128 columns of C by 16 or 32 rows and its partial
+ *                 is small) with a long K, where its measured cost model
+ *                 predicts a gain, and only into a workspace large enough
+ *                 (fp8_mm_workspace_size(..., 0) gives those bytes); larger
+ *                 problems are not split (on every shape measured on B200 the
+ *                 partials' round trip through L2 cost more than the shorter
+ *                 main loop saved);
  *                 1: no split; 2 .. 4: exactly that many splits.
- * workspace       NULL when no split is requested, else device memory,
+ * workspace       NULL (no split), else device memory,
  *                 16-byte aligned, of workspace_bytes >=
  *                 fp8_mm_workspace_size(..., split_k) bytes. Its first 4096
  *                 bytes are counters: they must be zero before the first call
@@ -226,8 +232,8 @@ FP8LITE_API fp8_status fp8_mm_ws(const uint8_t* a8, fp8_fmt fa, const uint8_t* b
                   void* stream);
 
 /* Workspace bytes fp8_mm_ws needs for this problem and split_k on the
- * current device: 0 when that call would not split (split_k 0 or 1), or for
- * arguments fp8_mm_ws rejects. */
+ * current device (split_k 0: for the library's own choice): 0 when that call
+ * would not split, or for arguments fp8_mm_ws rejects. */
 FP8LITE_API size_t fp8_mm_workspace_size(int64_t M, int64_t N, int64_t K, int64_t batch, fp8_layout layout,
                                          int32_t split_k);
 

@@ -131,7 +131,8 @@ def test_mm_workspace_size_and_alignment(fp8):
     assert fp8.fp8_mm_workspace_size(2048, 1024, 4096, 1, fp8.FP8_NT, 1) == 0
     # two splits: the counters plus at least two fp32 partials of the whole output
     assert fp8.fp8_mm_workspace_size(2048, 1024, 4096, 1, fp8.FP8_NT, 2) >= 4096 + 2 * 2048 * 1024 * 4
-    assert fp8.fp8_mm_workspace_size(1, 4096, 4096, 1, fp8.FP8_NT, 4) >= 4096 + 4 * 128 * 4096 * 4
+    # one row: swapped operands, partial tiles of 16 rows (M padded to 16, not 128)
+    assert fp8.fp8_mm_workspace_size(1, 4096, 4096, 1, fp8.FP8_NT, 4) == 4096 + 4 * 16 * 4096 * 4
     # too many tile halves for the counters, too few k-blocks, bad arguments
     assert fp8.fp8_mm_workspace_size(8192, 8192, 8192, 1, fp8.FP8_NT, 2) == 0
     assert fp8.fp8_mm_workspace_size(2048, 1024, 256, 1, fp8.FP8_NT, 4) == 0

@@ -224,3 +224,28 @@ def test_narrow_long_k_nt(g, M, N, K, bias_kind):
 
 def test_narrow_long_k_nt_batches(g):
     _full_check(g, NT, 384, 640, 1024, E4M3, E5M2, 1301, batch=2, bcast_b=True, pad_c=32, bias_kind=1)
+
+
+# Short problems (M <= 32, N >= 128, NT and NN) run with swapped operands: the
+# kernel computes C^T = B^T A^T on tiles of 128 columns of C by 16 or 32 rows
+# and writes C transposed. Every boundary of the 16/32-row tiles and of the
+# switch back to unswapped tiles at 33 rows, ragged N, both bias kinds,
+# batches with either operand broadcast, padded batch stride.
+
+@pytest.mark.parametrize("M,N,K,bias_kind", [(1, 128, 256, 0), (7, 1000, 384, 1), (16, 4096, 1024, 2),
+                                             (17, 256, 512, 1), (32, 640, 2048, 0), (33, 384, 256, 2),
+                                             (63, 1000, 512, 1), (64, 136, 128, 0)])
+def test_swapped_short_m_nt(g, M, N, K, bias_kind):
+    _full_check(g, NT, M, N, K, E4M3, E5M2, 1400 + M + N, bias_kind=bias_kind)
+
+
+@pytest.mark.parametrize("M,N,K,bias_kind", [(1, 144, 256, 1), (9, 1008, 384, 0), (16, 4096, 1024, 2),
+                                             (31, 640, 512, 1), (48, 384, 2048, 0), (64, 128, 128, 1)])
+def test_swapped_short_m_nn(g, M, N, K, bias_kind):
+    _full_check(g, NN, M, N, K, E5M2, E4M3, 1500 + M + N, bias_kind=bias_kind)
+
+
+@pytest.mark.parametrize("layout", [NT, NN])
+def test_swapped_batches(g, layout):
+    _full_check(g, layout, 12, 304, 256, E4M3, E4M3, 1601, batch=3, bcast_b=True, pad_c=24, bias_kind=1)
+    _full_check(g, layout, 40, 256, 384, E5M2, E4M3, 1602, batch=2, bcast_a=True)

@@ -159,3 +159,25 @@ def test_one_workspace_serves_a_sequence_and_graph_replay(g):
         assert not ws[:4096].any()
     del graph
     assert fp8.fp8_last_device_error() == fp8.FP8_OK
+
+
+@pytest.mark.parametrize("layout,M,N,K", [(NT, 1, 4096, 4096), (NN, 8, 4096, 4096), (NT, 16, 8192, 8192)])
+def test_automatic_split_of_short_problems(g, layout, M, N, K):
+    """split_k = 0 with a workspace: short problems with a long K split on
+    their own (the workspace size query says how much they need); the result
+    is the oracle's, bit-identical run to run, and fp8_mm (no workspace, no
+    split) agrees within the same bar."""
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    need = fp8.fp8_mm_workspace_size(M, N, K, 1, layout, 0)
+    assert need > 4096, "the automatic choice is expected to split this shape"
+    c = _case(layout, M, N, K, E4M3, E4M3, 1700 + M)
+    ws = g.workspace(need)
+    out = _run(g, c, layout, M, N, K, E4M3, E4M3, 1, ws, 0)
+    again = _run(g, c, layout, M, N, K, E4M3, E4M3, 1, ws, 0)
+    assert torch.equal(out.view(torch.int16), again.view(torch.int16))
+    assert not ws[:4096].any()
+    y, s = _oracle(c, layout, M, N, K, E4M3, E4M3, 1)
+    tol = oracle.tolerance(y, s)
+    g.assert_within(out.float().cpu().numpy().reshape(y.shape), y, tol, f"auto split {M}x{N}x{K}")
+    plain = _run(g, c, layout, M, N, K, E4M3, E4M3, 1, None, 0)
+    g.assert_within(plain.float().cpu().numpy().reshape(y.shape), y, tol, f"no split {M}x{N}x{K}")
