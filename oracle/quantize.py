@@ -28,6 +28,8 @@ Readings taken where the pages are silent:
   power-of-two rounding; a quotient that overflows fp32 is clamped to the
   largest finite fp32 value.
 * current scaling with amax = 0 or a non-finite amax uses scale 1.
+* a seeded ring call quantizes with the current scale of its input and then
+  folds that amax as usual (``DelayedRing.seed_step``).
 * the ring holds H = 16 entries, starts at hist = 0, idx = 0, scale = 1.
 * a window maximum that is 0 or non-finite keeps the previous scale.
 * the window includes the amax just written.
@@ -117,5 +119,18 @@ class DelayedRing:
         s = np.float32(self.scale)
         a = amax(x)
         q = quantize_with_scale(x, s, fmt)
+        self.fold(a, fmt)
+        return q, a, s
+
+    def seed_step(self, x, fmt: int):
+        """A seeded call: quantize x with its own current scale instead of
+        the ring's, then fold its amax like any call (the reading taken of the
+        ring's "seed" in ``astrai/extension/fp8.py @4dc5e923``, bullet on the
+        _ScaleRing objects with update/seed: a ring's first step can measure
+        its scale rather than start at the initial one).
+
+        Returns (codes, amax, scale used by this call).
+        """
+        q, a, s = quantize_current(x, fmt)
         self.fold(a, fmt)
         return q, a, s

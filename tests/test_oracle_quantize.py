@@ -152,3 +152,30 @@ def test_no_scale_ratio_leak_between_delayed_steps():
         y_bad, _ = oracle.mm(qx, E4M3, qw, E4M3, rx.scale, rw.scale, oracle.NT, 16, 8, 64)
         got = np.linalg.norm(y_bad[0]) / np.linalg.norm(true)
         assert abs(got / ratio - 1.0) < 0.1 and abs(ratio - 1.0) > 0.5
+
+
+def test_seeded_step_closed_forms():
+    """Fresh ring, x = [2, -1, 0.5, 0]: the seeded call scales by 448 / 2 = 224
+    (every product exactly representable in E4M3, so decoding the codes and
+    dividing by 224 gives x back exactly), writes 2 into hist[0], advances idx
+    to 1 and publishes 224; the next ordinary call uses 224. Seeding a ring
+    that already has history folds into hist[idx], not hist[0]."""
+    x = np.array([2.0, -1.0, 0.5, 0.0], np.float32)
+    r = oracle.DelayedRing()
+    q, a, s = r.seed_step(x, E4M3)
+    assert a == np.float32(2.0) and s == np.float32(224.0)
+    assert np.array_equal(oracle.decode_table(E4M3)[q] / np.float32(224.0), x)
+    assert r.hist[0] == np.float32(2.0) and not r.hist[1:].any() and r.idx == 1
+    assert r.scale == np.float32(224.0)
+    q2, a2, s2 = r.step(np.array([4.0], np.float32), E4M3)
+    assert s2 == np.float32(224.0) and r.scale == np.float32(112.0)  # window max 4 -> 448 / 4
+    # a ring with history: the seed folds at idx, and the window keeps the old maximum
+    r3 = oracle.DelayedRing()
+    r3.fold(np.float32(8.0), E4M3)
+    _, _, s3 = r3.seed_step(x, E4M3)
+    assert s3 == np.float32(224.0) and r3.hist[1] == np.float32(2.0) and r3.idx == 2
+    assert r3.scale == np.float32(56.0)  # 448 / max(8, 2)
+    # zero input: current scale 1, and the zero amax keeps the ring's scale
+    r4 = oracle.DelayedRing(3.0)
+    q4, a4, s4 = r4.seed_step(np.zeros(5, np.float32), E5M2)
+    assert s4 == np.float32(1.0) and a4 == 0 and r4.scale == np.float32(3.0) and not q4.any()
