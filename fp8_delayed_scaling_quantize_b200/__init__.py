@@ -25,6 +25,8 @@ FP8_ERR_CUDA = 4
 FP8_ERR_DEVICE_TIMEOUT = 5
 FP8_RING_HISTORY = 16
 FP8_RING_BYTES = 80
+FP8_IN_BF16, FP8_IN_F16, FP8_IN_F32 = 0, 1, 2
+FP8_QUANTIZE_SEED_RING = 1
 
 
 class Fp8Error(RuntimeError):
@@ -47,8 +49,11 @@ FP8_QUANTIZE_MAX_JOBS = 8
 class fp8_quantize_job(ctypes.Structure):
     """One job of fp8_quantize_many (pointers are device addresses)."""
     _fields_ = [("x", ctypes.c_void_p), ("n", ctypes.c_int64), ("fmt", ctypes.c_int32),
-                ("ring", ctypes.c_void_p), ("out8", ctypes.c_void_p), ("amax_out", ctypes.c_void_p),
-                ("scale_out", ctypes.c_void_p)]
+                ("dtype", ctypes.c_int32), ("ring", ctypes.c_void_p), ("out8", ctypes.c_void_p),
+                ("amax_out", ctypes.c_void_p), ("scale_out", ctypes.c_void_p)]
+
+
+assert ctypes.sizeof(fp8_quantize_job) == 56
 
 
 def _load():
@@ -63,6 +68,7 @@ def _load():
         "fp8_ring_get": (I, [P, P, P]),
         "fp8_ring_set": (I, [P, P, P]),
         "fp8_quantize": (I, [P, I64, I, P, P, P, P, P]),
+        "fp8_quantize_ex": (I, [P, I, I64, I, P, ctypes.c_uint32, P, P, P, P]),
         "fp8_mm": (I, [P, I, P, I, P, P, I, I64, I64, I64, I64, I64, I64, I64, P, P, I, P, P]),
         "fp8_last_device_error": (I, []),
         "fp8_selftest_wait_timeout": (I, [ctypes.c_uint32, P]),
@@ -138,11 +144,18 @@ def fp8_quantize(x, n, fmt, ring, out8, amax_out, scale_out, stream=None):
                                    _ptr(scale_out), _stream(stream)), "fp8_quantize")
 
 
+def fp8_quantize_ex(x, dtype, n, fmt, ring, flags, out8, amax_out, scale_out, stream=None):
+    return _check(lib.fp8_quantize_ex(_ptr(x), int(dtype), int(n), int(fmt), _ptr(ring), int(flags), _ptr(out8),
+                                      _ptr(amax_out), _ptr(scale_out), _stream(stream)), "fp8_quantize_ex")
+
+
 def fp8_quantize_many(jobs, stream=None):
-    """jobs: sequence of (x, n, fmt, ring, out8, amax_out, scale_out)."""
+    """jobs: sequence of (x, n, fmt, ring, out8, amax_out, scale_out[, dtype])."""
     arr = (fp8_quantize_job * max(len(jobs), 1))()
-    for i, (x, n, fmt, ring, out8, amax_out, scale_out) in enumerate(jobs):
-        arr[i] = fp8_quantize_job(_ptr(x), int(n), int(fmt), _ptr(ring), _ptr(out8), _ptr(amax_out),
+    for i, job in enumerate(jobs):
+        x, n, fmt, ring, out8, amax_out, scale_out = job[:7]
+        dtype = job[7] if len(job) > 7 else FP8_IN_BF16
+        arr[i] = fp8_quantize_job(_ptr(x), int(n), int(fmt), int(dtype), _ptr(ring), _ptr(out8), _ptr(amax_out),
                                   _ptr(scale_out))
     return _check(lib.fp8_quantize_many(ctypes.cast(arr, ctypes.c_void_p), len(jobs), _stream(stream)),
                   "fp8_quantize_many")

@@ -24,8 +24,15 @@
 //    next call (and for CUDA-graph replay) with no host involvement;
 //  * current: memset of the caller's amax word, an amax-only pass, then the
 //    quantize pass that derives the scale from that amax. For tensors that
-//    fit in L2 the second read is served from L2.
+//    fit in L2 the second read is served from L2;
+//  * seeded delayed call: the current-scaling passes, then block 0 folds the
+//    measured amax into the ring (astrai/extension/fp8.py @4dc5e923, bullet
+//    on the _ScaleRing objects with their update and seed);
+//  * inputs bf16, fp16 or fp32 (astrai/extension/fp8.py @f4c44ebf, bullet on
+//    the quantize kernel templated on the input type): every value widens to
+//    fp32 exactly; a unit is 8 elements (16 bytes of bf16/fp16, 32 of fp32).
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -38,7 +45,7 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kUnroll = 4;  // 16-byte units in flight per thread
 
-enum Mode { kDelayed = 0, kCurrentQuant = 1, kAmaxOnly = 2 };
+enum Mode { kDelayed = 0, kCurrentQuant = 1, kAmaxOnly = 2, kSeed = 3 };
 
 template <int FMT>
 __device__ __forceinline__ uint32_t cvt_pair(float lo, float hi) {
@@ -57,23 +64,71 @@ __device__ __forceinline__ uint32_t cvt_pair(float lo, float hi) {
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-template <int FMT>
-__device__ __forceinline__ uint32_t quant4(uint32_t w0, uint32_t w1, float s, float& m) {
-    const float a = bf_lo(w0), b = bf_hi(w0), c = bf_lo(w1), d = bf_hi(w1);
-    m = fmaxf(m, fabsf(a));
-    m = fmaxf(m, fabsf(b));
-    m = fmaxf(m, fabsf(c));
-    m = fmaxf(m, fabsf(d));
-    const uint32_t lo = cvt_pair<FMT>(__fmul_rn(a, s), __fmul_rn(b, s));
-    const uint32_t hi = cvt_pair<FMT>(__fmul_rn(c, s), __fmul_rn(d, s));
-    return lo | (hi << 16);
+// Eight consecutive input elements: 16 bytes of bf16 / fp16, 32 of fp32.
+struct Unit {
+    uint4 a, b;
+};
+
+template <int IN>
+__device__ __forceinline__ void load_unit(const void* x, int64_t i, Unit& u) {
+    if (IN == FP8_IN_F32) {
+        const uint4* p = static_cast<const uint4*>(x) + 2 * i;
+        u.a = __ldg(p);
+        u.b = __ldg(p + 1);
+    } else {
+        u.a = __ldg(static_cast<const uint4*>(x) + i);
+    }
 }
 
-__device__ __forceinline__ void amax4(uint32_t w0, uint32_t w1, float& m) {
-    m = fmaxf(m, fabsf(bf_lo(w0)));
-    m = fmaxf(m, fabsf(bf_hi(w0)));
-    m = fmaxf(m, fabsf(bf_lo(w1)));
-    m = fmaxf(m, fabsf(bf_hi(w1)));
+__device__ __forceinline__ float h_lo(uint32_t w) { return __half2float(__ushort_as_half(uint16_t(w & 0xFFFFu))); }
+__device__ __forceinline__ float h_hi(uint32_t w) { return __half2float(__ushort_as_half(uint16_t(w >> 16))); }
+
+// The unit's values in fp32 (exact for all three input types).
+template <int IN>
+__device__ __forceinline__ void unit_f32(const Unit& u, float (&f)[8]) {
+    const uint32_t w[4] = {u.a.x, u.a.y, u.a.z, u.a.w};
+    if (IN == FP8_IN_BF16) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = bf_lo(w[i]);
+            f[2 * i + 1] = bf_hi(w[i]);
+        }
+    } else if (IN == FP8_IN_F16) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = h_lo(w[i]);
+            f[2 * i + 1] = h_hi(w[i]);
+        }
+    } else {
+        const uint32_t v[4] = {u.b.x, u.b.y, u.b.z, u.b.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[i] = __uint_as_float(w[i]);
+            f[4 + i] = __uint_as_float(v[i]);
+        }
+    }
+}
+
+template <int IN>
+__device__ __forceinline__ float load_elem(const void* x, int64_t i) {
+    if (IN == FP8_IN_BF16) return __uint_as_float(uint32_t(static_cast<const uint16_t*>(x)[i]) << 16);
+    if (IN == FP8_IN_F16) return __half2float(static_cast<const __half*>(x)[i]);
+    return static_cast<const float*>(x)[i];
+}
+
+template <int FMT>
+__device__ __forceinline__ uint2 quant8(const float (&f)[8], float s, float& m) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
+    uint32_t p[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) p[i] = cvt_pair<FMT>(__fmul_rn(f[2 * i], s), __fmul_rn(f[2 * i + 1], s));
+    return make_uint2(p[0] | (p[1] << 16), p[2] | (p[3] << 16));
+}
+
+__device__ __forceinline__ void amax8(const float (&f)[8], float& m) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
 }
 
 __device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
@@ -99,12 +154,13 @@ __device__ __forceinline__ uint32_t block_max_bits(float m) {
 // The quantize pass of one tensor, run by block `blk` of the `nblk` blocks
 // given to it (a whole grid for fp8_quantize, a share of one for
 // fp8_quantize_many). s_scale is the block's shared scale slot.
-template <int FMT, int MODE>
-__device__ __forceinline__ void quantize_body(const uint16_t* __restrict__ x, int64_t n, uint8_t* __restrict__ out8,
+template <int FMT, int MODE, int IN>
+__device__ __forceinline__ void quantize_body(const void* __restrict__ x, int64_t n, uint8_t* __restrict__ out8,
                                               fp8_ring* ring, uint32_t* amax_acc, float* amax_out, float* scale_out,
                                               int blk, int nblk, float& s_scale) {
     const float fmax = fmt_max(FMT);
-    const uint4* xv = reinterpret_cast<const uint4*>(x);
+    // units in flight per thread: 64 bytes of input whatever the type
+    constexpr int U = IN == FP8_IN_F32 ? kUnroll / 2 : kUnroll;
     uint2* ov = reinterpret_cast<uint2*>(out8);
     const int64_t units = n >> 3;  // 8 elements per unit
     const int64_t tid = int64_t(blk) * kThreads + threadIdx.x;
@@ -113,11 +169,11 @@ __device__ __forceinline__ void quantize_body(const uint16_t* __restrict__ x, in
     // loads do not need it); for tensors of up to 2048 elements per thread
     // of the grid that is every load.
     int64_t base = tid;
-    uint4 v[kUnroll];
+    Unit v[U];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
+    for (int u = 0; u < U; ++u) {
         const int64_t i = base + u * stride;
-        if (i < units) v[u] = __ldg(xv + i);
+        if (i < units) load_unit<IN>(x, i, v[u]);
     }
     // One thread per block reads the scale (or the amax it comes from) and
     // shares it: thousands of warps loading one address would queue on a
@@ -127,7 +183,7 @@ __device__ __forceinline__ void quantize_body(const uint16_t* __restrict__ x, in
             float v;
             if (MODE == kDelayed) {
                 v = *reinterpret_cast<volatile float*>(&ring->scale);
-            } else {
+            } else {  // current scaling, also the seeded call: from the measured amax
                 const float a = __uint_as_float(*reinterpret_cast<volatile uint32_t*>(amax_acc));
                 v = (a > 0.0f && isfinite(a)) ? scale_from_amax(fmax, a) : 1.0f;
             }
@@ -141,49 +197,51 @@ __device__ __forceinline__ void quantize_body(const uint16_t* __restrict__ x, in
 
     while (base < units) {
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
+        for (int u = 0; u < U; ++u) {
             const int64_t i = base + u * stride;
             if (i < units) {
-                if (MODE == kAmaxOnly) {
-                    amax4(v[u].x, v[u].y, m);
-                    amax4(v[u].z, v[u].w, m);
-                } else {
-                    uint2 q;
-                    q.x = quant4<FMT>(v[u].x, v[u].y, s, m);
-                    q.y = quant4<FMT>(v[u].z, v[u].w, s, m);
-                    ov[i] = q;
-                }
+                float f[8];
+                unit_f32<IN>(v[u], f);
+                if (MODE == kAmaxOnly) amax8(f, m);
+                else                   ov[i] = quant8<FMT>(f, s, m);
             }
         }
-        base += stride * kUnroll;
+        base += stride * U;
         if (base >= units) break;
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
+        for (int u = 0; u < U; ++u) {
             const int64_t i = base + u * stride;
-            if (i < units) v[u] = __ldg(xv + i);
+            if (i < units) load_unit<IN>(x, i, v[u]);
         }
     }
     griddep_launch();  // the next kernel may start its prologue
     // ragged tail (n mod 8 elements): one thread, scalar
     if (tid == 0) {
         for (int64_t i = units << 3; i < n; ++i) {
-            const float a = __uint_as_float(uint32_t(x[i]) << 16);
+            const float a = load_elem<IN>(x, i);
             m = fmaxf(m, fabsf(a));
             if (MODE != kAmaxOnly) out8[i] = uint8_t(cvt_pair<FMT>(__fmul_rn(a, s), 0.0f));
         }
     }
 
-    const uint32_t bits = block_max_bits(m);
-    if (threadIdx.x != 0) return;
-    uint32_t* acc = MODE == kDelayed ? &ring->amax_bits : amax_acc;
-    if (bits != 0u) atomicMax(acc, bits);
-    if (MODE != kDelayed) return;
-
-    // Last-block election: every block publishes its amax, then takes a
-    // ticket with acquire-release semantics (its amax is visible before the
-    // ticket moves); the block holding the final ticket sees every amax.
-    const uint32_t ticket = atom_add_acq_rel(&ring->ticket, 1u);
-    if (ticket != uint32_t(nblk) - 1) return;
+    // the quantize pass of current scaling (and of a seeded call) already
+    // knows the amax: it came from the amax pass
+    if (MODE == kCurrentQuant) return;
+    if (MODE == kSeed) {
+        if (blk != 0 || threadIdx.x != 0) return;  // block 0 folds the amax into the ring
+    } else {
+        const uint32_t bits = block_max_bits(m);
+        if (threadIdx.x != 0) return;
+        uint32_t* acc = MODE == kDelayed ? &ring->amax_bits : amax_acc;
+        if (bits != 0u) atomicMax(acc, bits);
+        if (MODE != kDelayed) return;
+        // Last-block election: every block publishes its amax, then takes a
+        // ticket with acquire-release semantics (its amax is visible before
+        // the ticket moves); the block holding the final ticket sees every
+        // amax.
+        const uint32_t ticket = atom_add_acq_rel(&ring->ticket, 1u);
+        if (ticket != uint32_t(nblk) - 1) return;
+    }
     // The history and its index change only in this finalize, so they are
     // read together with the exchange of the accumulated amax: the 18
     // accesses leave at once and cost one round trip to L2.
@@ -192,7 +250,8 @@ __device__ __forceinline__ void quantize_body(const uint16_t* __restrict__ x, in
 #pragma unroll
     for (int i = 0; i < FP8_RING_HISTORY; ++i) h[i] = r->hist[i];
     const uint32_t idx = r->idx & (FP8_RING_HISTORY - 1);
-    const float a = __uint_as_float(atomicExch(&ring->amax_bits, 0u));
+    const float a = MODE == kDelayed ? __uint_as_float(atomicExch(&ring->amax_bits, 0u))
+                                     : __uint_as_float(*reinterpret_cast<volatile uint32_t*>(amax_acc));
     // the window's maximum over the 15 kept entries and the new amax
     float wmax = a;
 #pragma unroll
@@ -201,17 +260,19 @@ __device__ __forceinline__ void quantize_body(const uint16_t* __restrict__ x, in
     r->hist[idx] = a;
     if (wmax > 0.0f && isfinite(wmax)) r->scale = scale_from_amax(fmax, wmax);
     r->idx = (idx + 1) & (FP8_RING_HISTORY - 1);
-    if (amax_out) *amax_out = a;
-    r->ticket = 0u;  // ready for the next call (visible at the kernel boundary)
+    if (MODE == kDelayed) {
+        if (amax_out) *amax_out = a;
+        r->ticket = 0u;  // ready for the next call (visible at the kernel boundary)
+    }
 }
 
-template <int FMT, int MODE>
+template <int FMT, int MODE, int IN>
 __global__ void __launch_bounds__(kThreads)
-quantize_kernel(const uint16_t* __restrict__ x, int64_t n, uint8_t* __restrict__ out8,
+quantize_kernel(const void* __restrict__ x, int64_t n, uint8_t* __restrict__ out8,
                 fp8_ring* ring, uint32_t* amax_acc, float* amax_out, float* scale_out) {
     __shared__ float s_scale;
     griddep_wait();  // inputs and the ring come from earlier kernels
-    quantize_body<FMT, MODE>(x, n, out8, ring, amax_acc, amax_out, scale_out, blockIdx.x, gridDim.x, s_scale);
+    quantize_body<FMT, MODE, IN>(x, n, out8, ring, amax_acc, amax_out, scale_out, blockIdx.x, gridDim.x, s_scale);
 }
 
 // Several delayed-scaling quantizations in one launch: job j owns blocks
@@ -222,7 +283,8 @@ struct QuantJobs {
     int first[FP8_QUANTIZE_MAX_JOBS];
     int blocks[FP8_QUANTIZE_MAX_JOBS];
     int fmt[FP8_QUANTIZE_MAX_JOBS];
-    const uint16_t* x[FP8_QUANTIZE_MAX_JOBS];
+    int dtype[FP8_QUANTIZE_MAX_JOBS];
+    const void* x[FP8_QUANTIZE_MAX_JOBS];
     int64_t n[FP8_QUANTIZE_MAX_JOBS];
     fp8_ring* ring[FP8_QUANTIZE_MAX_JOBS];
     uint8_t* out8[FP8_QUANTIZE_MAX_JOBS];
@@ -236,12 +298,20 @@ __global__ void __launch_bounds__(kThreads) quantize_many_kernel(const __grid_co
     int j = 0;
     while (j + 1 < jobs.count && int(blockIdx.x) >= jobs.first[j + 1]) ++j;
     const int blk = int(blockIdx.x) - jobs.first[j];
-    if (jobs.fmt[j] == FP8_E4M3)
-        quantize_body<FP8_E4M3, kDelayed>(jobs.x[j], jobs.n[j], jobs.out8[j], jobs.ring[j], nullptr,
-                                          jobs.amax_out[j], jobs.scale_out[j], blk, jobs.blocks[j], s_scale);
-    else
-        quantize_body<FP8_E5M2, kDelayed>(jobs.x[j], jobs.n[j], jobs.out8[j], jobs.ring[j], nullptr,
-                                          jobs.amax_out[j], jobs.scale_out[j], blk, jobs.blocks[j], s_scale);
+#define FP8LITE_JOB(F, I)                                                                                        \
+    quantize_body<F, kDelayed, I>(jobs.x[j], jobs.n[j], jobs.out8[j], jobs.ring[j], nullptr, jobs.amax_out[j], \
+                                  jobs.scale_out[j], blk, jobs.blocks[j], s_scale)
+    const int dt = jobs.dtype[j];
+    if (jobs.fmt[j] == FP8_E4M3) {
+        if (dt == FP8_IN_BF16)     FP8LITE_JOB(FP8_E4M3, FP8_IN_BF16);
+        else if (dt == FP8_IN_F16) FP8LITE_JOB(FP8_E4M3, FP8_IN_F16);
+        else                       FP8LITE_JOB(FP8_E4M3, FP8_IN_F32);
+    } else {
+        if (dt == FP8_IN_BF16)     FP8LITE_JOB(FP8_E5M2, FP8_IN_BF16);
+        else if (dt == FP8_IN_F16) FP8LITE_JOB(FP8_E5M2, FP8_IN_F16);
+        else                       FP8LITE_JOB(FP8_E5M2, FP8_IN_F32);
+    }
+#undef FP8LITE_JOB
 }
 
 __global__ void ring_write_kernel(fp8_ring* ring, fp8_ring value) {
@@ -276,21 +346,36 @@ int grid_for(int64_t n) {
     return int(g < 1 ? 1 : g);
 }
 
-template <int FMT>
-fp8_status launch_quantize(const uint16_t* x, int64_t n, fp8_ring* ring, uint8_t* out8,
-                           float* amax_out, float* scale_out, cudaStream_t st) {
+template <int FMT, int IN>
+fp8_status launch_quantize(const void* x, int64_t n, fp8_ring* ring, bool seed, uint8_t* out8, float* amax_out,
+                           float* scale_out, cudaStream_t st) {
     const int grid = grid_for(n);
-    if (ring)
-        return launch_pdl(quantize_kernel<FMT, kDelayed>, grid, kThreads, 0, st, 1, x, n, out8, ring,
+    if (ring && !seed)
+        return launch_pdl(quantize_kernel<FMT, kDelayed, IN>, grid, kThreads, 0, st, 1, x, n, out8, ring,
                           (uint32_t*)nullptr, amax_out, scale_out);
     uint32_t* acc = reinterpret_cast<uint32_t*>(amax_out);
     if (cudaMemsetAsync(acc, 0, sizeof(uint32_t), st) != cudaSuccess) return FP8_ERR_CUDA;
-    if (launch_pdl(quantize_kernel<FMT, kAmaxOnly>, grid, kThreads, 0, st, 1, x, n, out8, (fp8_ring*)nullptr, acc,
-                   (float*)nullptr, (float*)nullptr) != FP8_OK)
+    if (launch_pdl(quantize_kernel<FMT, kAmaxOnly, IN>, grid, kThreads, 0, st, 1, x, n, out8, (fp8_ring*)nullptr,
+                   acc, (float*)nullptr, (float*)nullptr) != FP8_OK)
         return FP8_ERR_CUDA;
-    return launch_pdl(quantize_kernel<FMT, kCurrentQuant>, grid, kThreads, 0, st, 1, x, n, out8, (fp8_ring*)nullptr,
-                      acc, (float*)nullptr, scale_out);
+    if (seed)
+        return launch_pdl(quantize_kernel<FMT, kSeed, IN>, grid, kThreads, 0, st, 1, x, n, out8, ring, acc,
+                          (float*)nullptr, scale_out);
+    return launch_pdl(quantize_kernel<FMT, kCurrentQuant, IN>, grid, kThreads, 0, st, 1, x, n, out8,
+                      (fp8_ring*)nullptr, acc, (float*)nullptr, scale_out);
 }
+
+template <int FMT>
+fp8_status launch_quantize_in(fp8_dtype dtype, const void* x, int64_t n, fp8_ring* ring, bool seed, uint8_t* out8,
+                              float* amax_out, float* scale_out, cudaStream_t st) {
+    switch (dtype) {
+        case FP8_IN_BF16: return launch_quantize<FMT, FP8_IN_BF16>(x, n, ring, seed, out8, amax_out, scale_out, st);
+        case FP8_IN_F16:  return launch_quantize<FMT, FP8_IN_F16>(x, n, ring, seed, out8, amax_out, scale_out, st);
+        default:          return launch_quantize<FMT, FP8_IN_F32>(x, n, ring, seed, out8, amax_out, scale_out, st);
+    }
+}
+
+bool valid_dtype(int d) { return d == FP8_IN_BF16 || d == FP8_IN_F16 || d == FP8_IN_F32; }
 
 bool scale_ok(float s) { return s > 0.0f && s <= 3.402823466e38f; }
 
@@ -340,20 +425,28 @@ extern "C" fp8_status fp8_ring_set(fp8_ring* ring, const fp8_ring* host, void* s
     return launch_status();
 }
 
-extern "C" fp8_status fp8_quantize(const void* x, int64_t n, fp8_fmt fmt, fp8_ring* ring, uint8_t* out8,
-                                   float* amax_out, float* scale_out, void* stream) {
-    if (!valid_fmt(fmt)) return FP8_ERR_INVALID_ARG;
+extern "C" fp8_status fp8_quantize_ex(const void* x, fp8_dtype dtype, int64_t n, fp8_fmt fmt, fp8_ring* ring,
+                                      uint32_t flags, uint8_t* out8, float* amax_out, float* scale_out,
+                                      void* stream) {
+    if (!valid_fmt(fmt) || !valid_dtype(dtype)) return FP8_ERR_INVALID_ARG;
+    if ((flags & ~uint32_t(FP8_QUANTIZE_SEED_RING)) != 0u) return FP8_ERR_INVALID_ARG;
+    const bool seed = (flags & FP8_QUANTIZE_SEED_RING) != 0u;
+    if (seed && !ring) return FP8_ERR_INVALID_ARG;
     if (n < 0 || n >= (int64_t(1) << 40)) return FP8_ERR_INVALID_ARG;
     if (!scale_out) return FP8_ERR_INVALID_ARG;
     if (n > 0 && (!x || !out8)) return FP8_ERR_INVALID_ARG;
-    if (!ring && !amax_out) return FP8_ERR_INVALID_ARG;
+    if ((!ring || seed) && !amax_out) return FP8_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(out8, 16)) return FP8_ERR_ALIGNMENT;
     if (ring && !aligned(ring, 4)) return FP8_ERR_ALIGNMENT;
     if (!aligned(scale_out, 4) || !aligned(amax_out, 4)) return FP8_ERR_ALIGNMENT;
-    const uint16_t* xb = static_cast<const uint16_t*>(x);
     cudaStream_t st = as_stream(stream);
-    return fmt == FP8_E4M3 ? launch_quantize<FP8_E4M3>(xb, n, ring, out8, amax_out, scale_out, st)
-                           : launch_quantize<FP8_E5M2>(xb, n, ring, out8, amax_out, scale_out, st);
+    return fmt == FP8_E4M3 ? launch_quantize_in<FP8_E4M3>(dtype, x, n, ring, seed, out8, amax_out, scale_out, st)
+                           : launch_quantize_in<FP8_E5M2>(dtype, x, n, ring, seed, out8, amax_out, scale_out, st);
+}
+
+extern "C" fp8_status fp8_quantize(const void* x, int64_t n, fp8_fmt fmt, fp8_ring* ring, uint8_t* out8,
+                                   float* amax_out, float* scale_out, void* stream) {
+    return fp8_quantize_ex(x, FP8_IN_BF16, n, fmt, ring, 0u, out8, amax_out, scale_out, stream);
 }
 
 extern "C" fp8_status fp8_quantize_many(const fp8_quantize_job* jobs, int32_t count, void* stream) {
@@ -363,7 +456,7 @@ extern "C" fp8_status fp8_quantize_many(const fp8_quantize_job* jobs, int32_t co
     int total = 0;
     for (int j = 0; j < count; ++j) {
         const fp8_quantize_job& in = jobs[j];
-        if (!valid_fmt(in.fmt)) return FP8_ERR_INVALID_ARG;
+        if (!valid_fmt(in.fmt) || !valid_dtype(in.dtype)) return FP8_ERR_INVALID_ARG;
         if (in.n < 0 || in.n >= (int64_t(1) << 40)) return FP8_ERR_INVALID_ARG;
         if (!in.ring || !in.scale_out) return FP8_ERR_INVALID_ARG;
         if (in.n > 0 && (!in.x || !in.out8)) return FP8_ERR_INVALID_ARG;
@@ -375,7 +468,8 @@ extern "C" fp8_status fp8_quantize_many(const fp8_quantize_job* jobs, int32_t co
         q.blocks[j] = grid_for(in.n);
         total += q.blocks[j];
         q.fmt[j] = int(in.fmt);
-        q.x[j] = static_cast<const uint16_t*>(in.x);
+        q.dtype[j] = int(in.dtype);
+        q.x[j] = in.x;
         q.n[j] = in.n;
         q.ring[j] = in.ring;
         q.out8[j] = in.out8;

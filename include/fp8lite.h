@@ -26,7 +26,7 @@
 extern "C" {
 #endif
 
-#define FP8LITE_ABI_VERSION 1
+#define FP8LITE_ABI_VERSION 2
 
 /* Exported entry points (the library is built with hidden visibility). */
 #if defined(__GNUC__)
@@ -131,6 +131,32 @@ FP8LITE_API fp8_status fp8_quantize(const void* x, int64_t n, fp8_fmt fmt, fp8_r
                         uint8_t* out8, float* amax_out, float* scale_out,
                         void* stream);
 
+/* fp8_quantize for bf16, fp16 or fp32 input, with an optional seeded first
+ * call of a ring [fp8.py@f4c44ebf, bullet on the quantize kernel templated
+ * on the input type; fp8.py@4dc5e923, bullet on the _ScaleRing objects with
+ * their update and seed].
+ *
+ * dtype  the type of x: FP8_IN_BF16 (x is bf16[n]), FP8_IN_F16 (fp16[n]) or
+ *        FP8_IN_F32 (fp32[n]); every input value widens to fp32 exactly, so
+ *        the codes are those of the same values given as fp32.
+ * flags  0, or FP8_QUANTIZE_SEED_RING with a ring: instead of the ring's
+ *        current scale, this call measures amax(x) first, quantizes with
+ *        s = fmt_max / amax (1 if amax is 0 or not finite), and folds the amax
+ *        into the ring as a delayed call would (hist[idx] = amax, idx + 1, the
+ *        window's max publishes the next scale). Seeding a fresh ring (hist
+ *        all 0) so makes its next scale fmt_max / amax rather than leaving the
+ *        first step at the initial scale. Costs what current scaling costs
+ *        (a memset and two launches); amax_out is then REQUIRED (it is the
+ *        accumulator).
+ * Other arguments, results and errors as fp8_quantize (x 16-byte aligned
+ * whatever its type); FP8_ERR_INVALID_ARG also for an unknown dtype or flag
+ * and for FP8_QUANTIZE_SEED_RING without a ring. */
+typedef enum fp8_dtype { FP8_IN_BF16 = 0, FP8_IN_F16 = 1, FP8_IN_F32 = 2 } fp8_dtype;
+#define FP8_QUANTIZE_SEED_RING 1u
+FP8LITE_API fp8_status fp8_quantize_ex(const void* x, fp8_dtype dtype, int64_t n, fp8_fmt fmt, fp8_ring* ring,
+                        uint32_t flags, uint8_t* out8, float* amax_out, float* scale_out,
+                        void* stream);
+
 /* Several delayed-scaling quantizations in ONE launch, e.g. the weights of
  * all layers at the start of a training step, or a layer's x and W.
  * Each job is exactly an fp8_quantize call with a ring (same arguments, same
@@ -141,9 +167,10 @@ FP8LITE_API fp8_status fp8_quantize(const void* x, int64_t n, fp8_fmt fmt, fp8_r
  * FP8_ERR_INVALID_ARG for a bad count, a NULL ring or a ring used twice. */
 #define FP8_QUANTIZE_MAX_JOBS 8
 typedef struct fp8_quantize_job {
-    const void* x;     /* device bf16[n], 16-byte aligned */
+    const void* x;     /* device input of `dtype` [n], 16-byte aligned */
     int64_t n;         /* 0 <= n < 2^40 */
     int32_t fmt;       /* fp8_fmt */
+    int32_t dtype;     /* fp8_dtype of x (0 = bf16: a zero-filled job quantizes bf16) */
     fp8_ring* ring;    /* required */
     uint8_t* out8;     /* device uint8[n], 16-byte aligned */
     float* amax_out;   /* optional */

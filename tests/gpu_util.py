@@ -30,6 +30,17 @@ def quantize(x_dev, fmt, ring=None):
     return out, amax, scale
 
 
+def quantize_ex(x_dev, dtype, fmt, ring=None, flags=0):
+    """fp8_quantize_ex on a device tensor of any input type; returns
+    (codes, amax tensor[1], scale tensor[1])."""
+    n = x_dev.numel()
+    out = torch.empty(max(n, 1), dtype=torch.uint8, device=DEV)
+    amax = torch.full((1,), -1.0, dtype=torch.float32, device=DEV)
+    scale = torch.full((1,), -1.0, dtype=torch.float32, device=DEV)
+    fp8.fp8_quantize_ex(x_dev if n else None, dtype, n, fmt, ring, flags, out if n else None, amax, scale)
+    return out[:n], amax, scale
+
+
 def f32(t):
     return t.detach().float().cpu().numpy()
 

@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(fp8):
 
 
 def test_abi_version_and_status_strings(fp8):
-    assert fp8.fp8_abi_version() == 1
+    assert fp8.fp8_abi_version() == 2
     for code, name in [(0, "FP8_OK"), (1, "FP8_ERR_INVALID_ARG"), (2, "FP8_ERR_ALIGNMENT"),
                        (3, "FP8_ERR_UNSUPPORTED"), (4, "FP8_ERR_CUDA"), (5, "FP8_ERR_DEVICE_TIMEOUT")]:
         assert fp8.status_string(code) == name
@@ -115,13 +115,14 @@ def test_quantize_many_validation(fp8):
         arr = (fp8.fp8_quantize_job * max(len(jobs), 1))(*[fp8.fp8_quantize_job(*j) for j in jobs])
         return fp8.raw_status("fp8_quantize_many", ctypes.cast(arr, ctypes.c_void_p),
                               len(jobs) if count is None else count, None)
-    good = (A, 64, 0, S, A + 4096, None, S + 64)
+    good = (A, 64, 0, 0, S, A + 4096, None, S + 64)   # x, n, fmt, dtype, ring, out8, amax_out, scale_out
     assert status([good], count=0) == fp8.FP8_ERR_INVALID_ARG
     assert status([good] * 9) == fp8.FP8_ERR_INVALID_ARG
-    assert status([good, good]) == fp8.FP8_ERR_INVALID_ARG                    # one ring twice
-    assert status([(A, 64, 0, None, A + 4096, None, S + 64)]) == fp8.FP8_ERR_INVALID_ARG  # no ring
-    assert status([(A, 64, 5, S, A + 4096, None, S + 64)]) == fp8.FP8_ERR_INVALID_ARG     # bad fmt
-    assert status([(A + 2, 64, 0, S, A + 4096, None, S + 64)]) == fp8.FP8_ERR_ALIGNMENT
+    assert status([good, good]) == fp8.FP8_ERR_INVALID_ARG                       # one ring twice
+    assert status([(A, 64, 0, 0, None, A + 4096, None, S + 64)]) == fp8.FP8_ERR_INVALID_ARG  # no ring
+    assert status([(A, 64, 5, 0, S, A + 4096, None, S + 64)]) == fp8.FP8_ERR_INVALID_ARG     # bad fmt
+    assert status([(A, 64, 0, 3, S, A + 4096, None, S + 64)]) == fp8.FP8_ERR_INVALID_ARG     # bad dtype
+    assert status([(A + 2, 64, 0, 0, S, A + 4096, None, S + 64)]) == fp8.FP8_ERR_ALIGNMENT
     assert fp8.raw_status("fp8_quantize_many", None, 1, None) == fp8.FP8_ERR_INVALID_ARG
 
 
@@ -149,3 +150,16 @@ def test_mm_workspace_size_and_alignment(fp8):
         st = fp8.raw_status("fp8_mm_ws", A, 0, A, 0, S, S, 0, 16, 16, 16, 1, 256, 256, 256, None, None, 0, A,
                             A, 1 << 20, split_k, None)
         assert st == fp8.FP8_ERR_INVALID_ARG
+
+
+def test_quantize_ex_validation(fp8):
+    def st(x=A, dtype=0, n=64, fmt=0, ring=S, flags=0, out8=A + 4096, amax=S + 128, scale=S + 64):
+        return fp8.raw_status("fp8_quantize_ex", x, dtype, n, fmt, ring, flags, out8, amax, scale, None)
+    assert st(dtype=3) == fp8.FP8_ERR_INVALID_ARG
+    assert st(dtype=-1) == fp8.FP8_ERR_INVALID_ARG
+    assert st(flags=2) == fp8.FP8_ERR_INVALID_ARG                        # unknown flag
+    assert st(ring=None, flags=fp8.FP8_QUANTIZE_SEED_RING) == fp8.FP8_ERR_INVALID_ARG  # seed needs a ring
+    assert st(flags=fp8.FP8_QUANTIZE_SEED_RING, amax=None) == fp8.FP8_ERR_INVALID_ARG  # seed needs amax_out
+    assert st(ring=None, amax=None) == fp8.FP8_ERR_INVALID_ARG           # current scaling needs amax_out
+    assert st(x=A + 4, dtype=2) == fp8.FP8_ERR_ALIGNMENT                 # fp32 input still 16-byte aligned
+    assert st(fmt=7) == fp8.FP8_ERR_INVALID_ARG

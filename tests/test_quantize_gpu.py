@@ -215,3 +215,115 @@ def test_quantize_many_matches_the_oracle_per_job(g):
             hist, rs, idx, acc, ticket = g.ring_state(rings[j])
             assert np.array_equal(hist, refs[j].hist) and rs == refs[j].scale and idx == refs[j].idx
             assert acc == 0 and ticket == 0
+
+
+# ---------------------------------------------------- fp16 / fp32 inputs ---
+
+@pytest.mark.parametrize("fmt", [E4M3, E5M2])
+def test_every_f16_pattern_under_many_scales(g, fmt):
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    xs = W.f16_bit_patterns()
+    xf = xs.float().numpy()
+    nan = np.isnan(xf)
+    xd = xs.cuda()
+    for s in [1.0, 3.5, 2.0 ** -10, 1.0e4, 2.0 ** 20, 0.1]:
+        s32 = np.float32(s)
+        ring = g.new_ring()
+        host = fp8.fp8_ring()
+        host.scale = float(s32)
+        fp8.fp8_ring_set(ring, host)
+        q, amax, scale = g.quantize_ex(xd, fp8.FP8_IN_F16, fmt, ring)
+        got = g.codes(q)
+        want = oracle.quantize_with_scale(xf, s32, fmt)
+        assert np.array_equal(got[~nan], want[~nan]), f"scale {s}"
+        assert all(_nan_code(int(c), fmt) for c in got[nan])
+        assert g.f32(scale)[0] == s32 and g.f32(amax)[0] == oracle.amax(xf)
+
+
+@pytest.mark.parametrize("fmt", [E4M3, E5M2])
+def test_f32_inputs_over_the_whole_range(g, fmt):
+    """fp32 values from subnormal to FLT_MAX with +-0 and +-inf mixed in:
+    delayed (a given scale) and current scaling, on the finite-only copy too
+    (so that the measured scale is not the amax = inf fallback)."""
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    n = (1 << 20) + 5
+    x = W.f32_mixed(n, 6000 + fmt)
+    xf = x.numpy()
+    for s in [1.0, 2.0 ** -60, 2.0 ** 40, 7.0]:
+        s32 = np.float32(s)
+        ring = g.new_ring()
+        host = fp8.fp8_ring()
+        host.scale = float(s32)
+        fp8.fp8_ring_set(ring, host)
+        q, amax, scale = g.quantize_ex(x.cuda(), fp8.FP8_IN_F32, fmt, ring)
+        assert np.array_equal(g.codes(q), oracle.quantize_with_scale(xf, s32, fmt)), f"scale {s}"
+        assert g.f32(amax)[0] == oracle.amax(xf) == np.inf
+    finite = x.clone()
+    finite[~torch.isfinite(finite)] = 0.0
+    for t in (x, finite):
+        q, amax, scale = g.quantize_ex(t.cuda(), fp8.FP8_IN_F32, fmt, None)
+        want, a, s = oracle.quantize_current(t.numpy(), fmt)
+        assert np.array_equal(g.codes(q), want)
+        assert g.f32(amax)[0] == a and g.f32(scale)[0] == s
+
+
+@pytest.mark.parametrize("dtype", [1, 2])
+@pytest.mark.parametrize("n", [1, 7, 9, 1000, 4096 * 37 + 5])
+def test_f16_f32_ragged_sizes(g, dtype, n):
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    x = W.bf16_normal((n,), 0.7, 9100 + n).float()
+    x = x.to(torch.float16) if dtype == fp8.FP8_IN_F16 else x * 1.0001
+    q, amax, scale = g.quantize_ex(x.cuda(), dtype, E4M3, None)
+    want, a, s = oracle.quantize_current(x.float().numpy(), E4M3)
+    assert np.array_equal(g.codes(q), want) and g.f32(amax)[0] == a and g.f32(scale)[0] == s
+    ring = g.new_ring(2.0)
+    ref = oracle.DelayedRing(2.0)
+    for _ in range(2):
+        q, amax, scale = g.quantize_ex(x.cuda(), dtype, E5M2, ring)
+        want, a, s = ref.step(x.float().numpy(), E5M2)
+        assert np.array_equal(g.codes(q), want) and g.f32(scale)[0] == s
+    hist, rs, idx, _, _ = g.ring_state(ring)
+    assert np.array_equal(hist, ref.hist) and rs == ref.scale and idx == ref.idx
+
+
+def test_quantize_many_mixed_input_types(g):
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    xs = [W.bf16_normal((70001,), 0.5, 9201), W.bf16_normal((4096 * 9,), 2.0, 9202).float().to(torch.float16),
+          W.f32_mixed(1 << 18, 9203), W.bf16_normal((33,), 0.1, 9204).float()]
+    dts = [fp8.FP8_IN_BF16, fp8.FP8_IN_F16, fp8.FP8_IN_F32, fp8.FP8_IN_F32]
+    fmts = [E4M3, E5M2, E4M3, E5M2]
+    rings = [g.new_ring(1.5) for _ in xs]
+    refs = [oracle.DelayedRing(1.5) for _ in xs]
+    outs = [torch.empty(x.numel(), dtype=torch.uint8, device="cuda") for x in xs]
+    scs = [torch.empty(1, device="cuda") for _ in xs]
+    xd = [x.cuda() for x in xs]
+    for _ in range(2):
+        fp8.fp8_quantize_many([(xd[j], xs[j].numel(), fmts[j], rings[j], outs[j], None, scs[j], dts[j])
+                               for j in range(len(xs))])
+        for j, x in enumerate(xs):
+            want, a, s = refs[j].step(x.float().numpy(), fmts[j])
+            assert np.array_equal(g.codes(outs[j]), want), j
+            assert g.f32(scs[j])[0] == s
+            hist, rs, idx, acc, ticket = g.ring_state(rings[j])
+            assert np.array_equal(hist, refs[j].hist) and rs == refs[j].scale and acc == 0 and ticket == 0
+
+
+@pytest.mark.parametrize("dtype", [0, 1, 2])
+def test_seeded_first_call(g, dtype):
+    """A fresh ring's seeded call quantizes with the input's own scale and
+    folds its amax; the ordinary calls after it follow the oracle's ring."""
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    torch_dt = {0: torch.bfloat16, 1: torch.float16, 2: torch.float32}[dtype]
+    ring = g.new_ring()
+    ref = oracle.DelayedRing()
+    for step in range(4):
+        x = (W.bf16_normal((300001,), 0.03, 9300 + step).float() * (step + 1)).to(torch_dt)
+        flags = fp8.FP8_QUANTIZE_SEED_RING if step == 0 else 0
+        q, amax, scale = g.quantize_ex(x.cuda(), dtype, E4M3, ring, flags)
+        xf = x.float().numpy()
+        want, a, s = ref.seed_step(xf, E4M3) if step == 0 else ref.step(xf, E4M3)
+        assert np.array_equal(g.codes(q), want), step
+        assert g.f32(scale)[0] == s and g.f32(amax)[0] == a, step
+        hist, rs, idx, acc, ticket = g.ring_state(ring)
+        assert np.array_equal(hist, ref.hist) and rs == ref.scale and idx == ref.idx, step
+        assert acc == 0 and ticket == 0

@@ -23,6 +23,8 @@ Workloads (the shapes and distributions of the FP8 linear-layer path):
    1024x1536x2048 and decode shapes M in {1, 8} x N = 4096 x K = 4096.
 5. batched E4M3 GEMMs: 64 x 512^3 independent, and 8 x 1024x2048x2048 with
    B broadcast (batch stride 0).
+6. quantize inputs of the other types: every fp16 bit pattern, and fp32
+   values over the whole fp32 range with the special values mixed in.
 """
 
 import torch
@@ -64,6 +66,29 @@ def fp8_codes(shape, fmt: int, seed: int) -> torch.Tensor:
 def bf16_bit_patterns() -> torch.Tensor:
     """Every one of the 65536 bf16 bit patterns, as a bf16 tensor."""
     return torch.arange(0, 65536, dtype=torch.int32).to(torch.int16).view(torch.bfloat16)
+
+
+def f16_bit_patterns() -> torch.Tensor:
+    """Every one of the 65536 fp16 bit patterns, as an fp16 tensor."""
+    return torch.arange(0, 65536, dtype=torch.int32).to(torch.int16).view(torch.float16)
+
+
+def f32_mixed(n: int, seed: int) -> torch.Tensor:
+    """fp32 tensor of n values spread over the whole fp32 range: normal draws
+    scaled by 2^e with e ~ U{-140, ..., 130} (so subnormals, values that
+    overflow any FP8 scale and everything between occur), random signs, and
+    every 97th value replaced by one of +-0, +-inf, the smallest subnormal
+    and the largest finite fp32."""
+    g = _gen(seed)
+    x = torch.randn(n, generator=g, dtype=torch.float64)
+    e = torch.randint(-140, 131, (n,), generator=g).to(torch.float64)
+    v = (x * torch.pow(2.0, e)).to(torch.float32)
+    special = torch.tensor([0.0, -0.0, float("inf"), -float("inf"), 1.401298464324817e-45,
+                            -1.401298464324817e-45, 3.4028234663852886e38, -3.4028234663852886e38],
+                           dtype=torch.float32)
+    idx = torch.arange(0, n, 97)
+    v[idx] = special[torch.arange(len(idx)) % len(special)]
+    return v
 
 
 # ------------------------------------------------------------- workloads ---
