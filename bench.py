@@ -736,6 +736,18 @@ def run_kernel(args):
         call = lambda i: fp8.fp8_mm_ws(sets[i % 2][0], E4M3, sets[i % 2][1], E4M3, sa, sa, layout, M, N, K, 1, 0, 0,
                                        0, None, None, 0, out, ws, args.split_k if need else 0, stream=st)
         units = 2.0 * M * N * K
+    elif args.kernel == "quantize_2d":
+        # both orientations of a bf16 [rows, cols] tensor from one pass, delayed
+        rows, cols = (int(v) for v in args.shape.split("x"))
+        xs = [W.bf16_normal((rows, cols), 1.0, 9500 + i).cuda() for i in range(2)]
+        q = torch.empty(rows * cols, dtype=torch.uint8, device="cuda")
+        qt = torch.empty(rows * cols, dtype=torch.uint8, device="cuda")
+        ring = torch.empty(20, dtype=torch.int32, device="cuda")
+        fp8.fp8_ring_init(ring, 1.0)
+        sc = torch.empty(1, device="cuda")
+        am = torch.empty(1, device="cuda")
+        call = lambda i: fp8.fp8_quantize_2d(xs[i % 2], 0, rows, cols, E4M3, ring, 0, 2, q, qt, am, sc, stream=st)
+        units = 4.0 * rows * cols  # 2 bytes read, 1 + 1 written per element
     elif args.kernel == "quantize_many":
         # the linear stack's step-start launch: every weight and the first x
         sizes = [d_out * d_in for _, d_in, d_out in W.LINEARS] + [W.TOKENS * W.LINEARS[0][1]]
@@ -781,7 +793,8 @@ def run_kernel(args):
                           "peak_source": src}))
     else:
         ach = units / (us * 1e-6) / 1e9
-        print(json.dumps({"kernel": args.kernel, "n": int(units / 3), "us": round(us, 2), "gbs": round(ach, 1),
+        n_el = int(units / 4) if args.kernel == "quantize_2d" else int(units / 3)
+        print(json.dumps({"kernel": args.kernel, "n": n_el, "us": round(us, 2), "gbs": round(ach, 1),
                           "frac_hbm": round(ach / hbm, 4), "peak": hbm, "peak_source": src}))
 
 
@@ -800,7 +813,8 @@ def main():
     ap.add_argument("--no-compare", action="store_true", help="skip the bf16 / autograd comparison")
     ap.add_argument("--breakdown-reps", type=int, default=20)
     ap.add_argument("--e2e-steps", type=int, default=10)
-    ap.add_argument("--kernel", choices=["gemm", "quantize", "quantize_many", "cublaslt"], help="single-kernel mode")
+    ap.add_argument("--kernel", choices=["gemm", "quantize", "quantize_many", "quantize_2d", "cublaslt"],
+                    help="single-kernel mode")
     ap.add_argument("--shape", default="8192x8192x8192", help="MxNxK for gemm, n for quantize")
     ap.add_argument("--layout", default="NT", choices=["NT", "NN", "TN"])
     args = ap.parse_args()

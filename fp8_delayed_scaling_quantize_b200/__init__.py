@@ -26,6 +26,7 @@ FP8_ERR_DEVICE_TIMEOUT = 5
 FP8_RING_HISTORY = 16
 FP8_RING_BYTES = 80
 FP8_IN_BF16, FP8_IN_F16, FP8_IN_F32 = 0, 1, 2
+FP8_QL_ROW, FP8_QL_COL, FP8_QL_BOTH = 0, 1, 2
 FP8_QUANTIZE_SEED_RING = 1
 
 
@@ -69,6 +70,7 @@ def _load():
         "fp8_ring_set": (I, [P, P, P]),
         "fp8_quantize": (I, [P, I64, I, P, P, P, P, P]),
         "fp8_quantize_ex": (I, [P, I, I64, I, P, ctypes.c_uint32, P, P, P, P]),
+        "fp8_quantize_2d": (I, [P, I, I64, I64, I, P, ctypes.c_uint32, I, P, P, P, P, P]),
         "fp8_mm": (I, [P, I, P, I, P, P, I, I64, I64, I64, I64, I64, I64, I64, P, P, I, P, P]),
         "fp8_last_device_error": (I, []),
         "fp8_selftest_wait_timeout": (I, [ctypes.c_uint32, P]),
@@ -147,6 +149,13 @@ def fp8_quantize(x, n, fmt, ring, out8, amax_out, scale_out, stream=None):
 def fp8_quantize_ex(x, dtype, n, fmt, ring, flags, out8, amax_out, scale_out, stream=None):
     return _check(lib.fp8_quantize_ex(_ptr(x), int(dtype), int(n), int(fmt), _ptr(ring), int(flags), _ptr(out8),
                                       _ptr(amax_out), _ptr(scale_out), _stream(stream)), "fp8_quantize_ex")
+
+
+def fp8_quantize_2d(x, dtype, rows, cols, fmt, ring, flags, layout, out8, out8_t, amax_out, scale_out,
+                    stream=None):
+    return _check(lib.fp8_quantize_2d(_ptr(x), int(dtype), int(rows), int(cols), int(fmt), _ptr(ring), int(flags),
+                                      int(layout), _ptr(out8), _ptr(out8_t), _ptr(amax_out), _ptr(scale_out),
+                                      _stream(stream)), "fp8_quantize_2d")
 
 
 def fp8_quantize_many(jobs, stream=None):

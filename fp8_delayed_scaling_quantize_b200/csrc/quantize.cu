@@ -151,79 +151,13 @@ __device__ __forceinline__ uint32_t block_max_bits(float m) {
     return bits;
 }
 
-// The quantize pass of one tensor, run by block `blk` of the `nblk` blocks
-// given to it (a whole grid for fp8_quantize, a share of one for
-// fp8_quantize_many). s_scale is the block's shared scale slot.
-template <int FMT, int MODE, int IN>
-__device__ __forceinline__ void quantize_body(const void* __restrict__ x, int64_t n, uint8_t* __restrict__ out8,
-                                              fp8_ring* ring, uint32_t* amax_acc, float* amax_out, float* scale_out,
-                                              int blk, int nblk, float& s_scale) {
+// The end of a block's pass: its amax goes to the accumulator (amax pass,
+// delayed call), and the ring is finalized by the last block of a delayed call
+// or by block 0 of a seeded call. m: this thread's amax.
+template <int FMT, int MODE>
+__device__ __forceinline__ void finish_block(float m, fp8_ring* ring, uint32_t* amax_acc, float* amax_out, int blk,
+                                             int nblk) {
     const float fmax = fmt_max(FMT);
-    // units in flight per thread: 64 bytes of input whatever the type
-    constexpr int U = IN == FP8_IN_F32 ? kUnroll / 2 : kUnroll;
-    uint2* ov = reinterpret_cast<uint2*>(out8);
-    const int64_t units = n >> 3;  // 8 elements per unit
-    const int64_t tid = int64_t(blk) * kThreads + threadIdx.x;
-    const int64_t stride = int64_t(nblk) * kThreads;
-    // The first round of input loads leaves before the scale is known (the
-    // loads do not need it); for tensors of up to 2048 elements per thread
-    // of the grid that is every load.
-    int64_t base = tid;
-    Unit v[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-        const int64_t i = base + u * stride;
-        if (i < units) load_unit<IN>(x, i, v[u]);
-    }
-    // One thread per block reads the scale (or the amax it comes from) and
-    // shares it: thousands of warps loading one address would queue on a
-    // single L2 line.
-    if (MODE != kAmaxOnly) {
-        if (threadIdx.x == 0) {
-            float v;
-            if (MODE == kDelayed) {
-                v = *reinterpret_cast<volatile float*>(&ring->scale);
-            } else {  // current scaling, also the seeded call: from the measured amax
-                const float a = __uint_as_float(*reinterpret_cast<volatile uint32_t*>(amax_acc));
-                v = (a > 0.0f && isfinite(a)) ? scale_from_amax(fmax, a) : 1.0f;
-            }
-            s_scale = v;
-            if (blk == 0) *scale_out = v;
-        }
-        __syncthreads();
-    }
-    const float s = MODE == kAmaxOnly ? 1.0f : s_scale;
-    float m = 0.0f;
-
-    while (base < units) {
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t i = base + u * stride;
-            if (i < units) {
-                float f[8];
-                unit_f32<IN>(v[u], f);
-                if (MODE == kAmaxOnly) amax8(f, m);
-                else                   ov[i] = quant8<FMT>(f, s, m);
-            }
-        }
-        base += stride * U;
-        if (base >= units) break;
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t i = base + u * stride;
-            if (i < units) load_unit<IN>(x, i, v[u]);
-        }
-    }
-    griddep_launch();  // the next kernel may start its prologue
-    // ragged tail (n mod 8 elements): one thread, scalar
-    if (tid == 0) {
-        for (int64_t i = units << 3; i < n; ++i) {
-            const float a = load_elem<IN>(x, i);
-            m = fmaxf(m, fabsf(a));
-            if (MODE != kAmaxOnly) out8[i] = uint8_t(cvt_pair<FMT>(__fmul_rn(a, s), 0.0f));
-        }
-    }
-
     // the quantize pass of current scaling (and of a seeded call) already
     // knows the amax: it came from the amax pass
     if (MODE == kCurrentQuant) return;
@@ -266,6 +200,86 @@ __device__ __forceinline__ void quantize_body(const void* __restrict__ x, int64_
     }
 }
 
+// The scale a quantize pass uses, read by one thread per block and shared
+// (thousands of warps loading one address would queue on a single L2 line):
+// the ring's for a delayed call, fmt_max / amax from the amax pass otherwise.
+// Block 0 also reports it in scale_out.
+template <int FMT, int MODE>
+__device__ __forceinline__ float read_scale(fp8_ring* ring, uint32_t* amax_acc, float* scale_out, int blk,
+                                            float& s_scale) {
+    if (threadIdx.x == 0) {
+        float v;
+        if (MODE == kDelayed) {
+            v = *reinterpret_cast<volatile float*>(&ring->scale);
+        } else {  // current scaling, also the seeded call: from the measured amax
+            const float a = __uint_as_float(*reinterpret_cast<volatile uint32_t*>(amax_acc));
+            v = (a > 0.0f && isfinite(a)) ? scale_from_amax(fmt_max(FMT), a) : 1.0f;
+        }
+        s_scale = v;
+        if (blk == 0) *scale_out = v;
+    }
+    __syncthreads();
+    return s_scale;
+}
+
+// The quantize pass of one tensor, run by block `blk` of the `nblk` blocks
+// given to it (a whole grid for fp8_quantize, a share of one for
+// fp8_quantize_many). s_scale is the block's shared scale slot.
+template <int FMT, int MODE, int IN>
+__device__ __forceinline__ void quantize_body(const void* __restrict__ x, int64_t n, uint8_t* __restrict__ out8,
+                                              fp8_ring* ring, uint32_t* amax_acc, float* amax_out, float* scale_out,
+                                              int blk, int nblk, float& s_scale) {
+    // units in flight per thread: 64 bytes of input whatever the type
+    constexpr int U = IN == FP8_IN_F32 ? kUnroll / 2 : kUnroll;
+    uint2* ov = reinterpret_cast<uint2*>(out8);
+    const int64_t units = n >> 3;  // 8 elements per unit
+    const int64_t tid = int64_t(blk) * kThreads + threadIdx.x;
+    const int64_t stride = int64_t(nblk) * kThreads;
+    // The first round of input loads leaves before the scale is known (the
+    // loads do not need it); for tensors of up to 2048 elements per thread
+    // of the grid that is every load.
+    int64_t base = tid;
+    Unit v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int64_t i = base + u * stride;
+        if (i < units) load_unit<IN>(x, i, v[u]);
+    }
+    const float s = MODE == kAmaxOnly ? 1.0f : read_scale<FMT, MODE>(ring, amax_acc, scale_out, blk, s_scale);
+    float m = 0.0f;
+
+    while (base < units) {
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = base + u * stride;
+            if (i < units) {
+                float f[8];
+                unit_f32<IN>(v[u], f);
+                if (MODE == kAmaxOnly) amax8(f, m);
+                else                   ov[i] = quant8<FMT>(f, s, m);
+            }
+        }
+        base += stride * U;
+        if (base >= units) break;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = base + u * stride;
+            if (i < units) load_unit<IN>(x, i, v[u]);
+        }
+    }
+    griddep_launch();  // the next kernel may start its prologue
+    // ragged tail (n mod 8 elements): one thread, scalar
+    if (tid == 0) {
+        for (int64_t i = units << 3; i < n; ++i) {
+            const float a = load_elem<IN>(x, i);
+            m = fmaxf(m, fabsf(a));
+            if (MODE != kAmaxOnly) out8[i] = uint8_t(cvt_pair<FMT>(__fmul_rn(a, s), 0.0f));
+        }
+    }
+
+    finish_block<FMT, MODE>(m, ring, amax_acc, amax_out, blk, nblk);
+}
+
 template <int FMT, int MODE, int IN>
 __global__ void __launch_bounds__(kThreads)
 quantize_kernel(const void* __restrict__ x, int64_t n, uint8_t* __restrict__ out8,
@@ -273,6 +287,77 @@ quantize_kernel(const void* __restrict__ x, int64_t n, uint8_t* __restrict__ out
     __shared__ float s_scale;
     griddep_wait();  // inputs and the ring come from earlier kernels
     quantize_body<FMT, MODE, IN>(x, n, out8, ring, amax_acc, amax_out, scale_out, blockIdx.x, gridDim.x, s_scale);
+}
+
+// Quantize of a [rows, cols] tensor that also writes the transposed codes
+// [cols, rows] (LAYOUT FP8_QL_COL: only those; FP8_QL_BOTH: both, from one read
+// of the input). A block walks 64 x 64 tiles: each thread quantizes one 8-element
+// unit of a row (exactly as the flat kernel does, so both orientations hold
+// the same bytes), writes it to the row-major codes, and drops its 8 codes into a
+// shared-memory tile column; after a barrier each thread reads 8 consecutive
+// codes of a tile row, which are 8 consecutive rows of one input column, and
+// writes them to the transposed codes. rows and cols are multiples of 8.
+constexpr int kTile = 64;
+constexpr int kTileStride = kTile + 4;  // bytes per shared tile row: 4-byte reads, 2-way conflicts on the writes
+
+template <int FMT, int MODE, int IN, int LAYOUT>
+__global__ void __launch_bounds__(kThreads)
+quantize2d_kernel(const void* __restrict__ x, int64_t rows, int64_t cols, uint8_t* __restrict__ out8,
+                  uint8_t* __restrict__ out8_t, fp8_ring* ring, uint32_t* amax_acc, float* amax_out,
+                  float* scale_out) {
+    static_assert(kThreads == kTile * kTile / 8, "one unit per thread and tile");
+    __shared__ float s_scale;
+    __shared__ __align__(16) uint8_t tile[kTile][kTileStride];
+    griddep_wait();
+    const int64_t trows = (rows + kTile - 1) / kTile, tcols = (cols + kTile - 1) / kTile;
+    const int64_t tiles = trows * tcols;
+    const int lr = threadIdx.x >> 3;        // tile row this thread loads
+    const int lc = (threadIdx.x & 7) * 8;   // its first tile column
+    const int oc = threadIdx.x >> 3;        // tile column (transposed row) it writes
+    const int orow = (threadIdx.x & 7) * 8; // its first tile row there
+    // the first tile's load leaves before the scale is known
+    int64_t t = blockIdx.x;
+    Unit v;
+    int64_t r0 = 0, c0 = 0;
+    bool have = false;
+    if (t < tiles) {
+        r0 = (t / tcols) * kTile;
+        c0 = (t % tcols) * kTile;
+        have = r0 + lr < rows && c0 + lc < cols;
+        if (have) load_unit<IN>(x, ((r0 + lr) * cols + c0 + lc) >> 3, v);
+    }
+    const float s = read_scale<FMT, MODE>(ring, amax_acc, scale_out, blockIdx.x, s_scale);
+    float m = 0.0f;
+    while (t < tiles) {
+        uint2 q = make_uint2(0u, 0u);
+        if (have) {
+            float f[8];
+            unit_f32<IN>(v, f);
+            q = quant8<FMT>(f, s, m);
+            if (LAYOUT == FP8_QL_BOTH) *reinterpret_cast<uint2*>(out8 + (r0 + lr) * cols + c0 + lc) = q;
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            tile[lc + k][lr] = uint8_t(q.x >> (8 * k));
+            tile[lc + 4 + k][lr] = uint8_t(q.y >> (8 * k));
+        }
+        __syncthreads();
+        if (c0 + oc < cols && r0 + orow < rows) {
+            const uint32_t w0 = *reinterpret_cast<const uint32_t*>(&tile[oc][orow]);
+            const uint32_t w1 = *reinterpret_cast<const uint32_t*>(&tile[oc][orow + 4]);
+            *reinterpret_cast<uint2*>(out8_t + (c0 + oc) * rows + r0 + orow) = make_uint2(w0, w1);
+        }
+        t += gridDim.x;
+        if (t < tiles) {  // the next tile's load, then the barrier that frees the shared tile
+            r0 = (t / tcols) * kTile;
+            c0 = (t % tcols) * kTile;
+            have = r0 + lr < rows && c0 + lc < cols;
+            if (have) load_unit<IN>(x, ((r0 + lr) * cols + c0 + lc) >> 3, v);
+        }
+        __syncthreads();
+    }
+    griddep_launch();
+    finish_block<FMT, MODE>(m, ring, amax_acc, amax_out, blockIdx.x, gridDim.x);
 }
 
 // Several delayed-scaling quantizations in one launch: job j owns blocks
@@ -377,6 +462,45 @@ fp8_status launch_quantize_in(fp8_dtype dtype, const void* x, int64_t n, fp8_rin
 
 bool valid_dtype(int d) { return d == FP8_IN_BF16 || d == FP8_IN_F16 || d == FP8_IN_F32; }
 
+template <int FMT, int IN, int LAYOUT>
+fp8_status launch_quantize_2d(const void* x, int64_t rows, int64_t cols, fp8_ring* ring, bool seed, uint8_t* out8,
+                              uint8_t* out8_t, float* amax_out, float* scale_out, cudaStream_t st) {
+    const int64_t tiles = ((rows + kTile - 1) / kTile) * ((cols + kTile - 1) / kTile);
+    const int64_t cap = int64_t(sm_count()) * (2048 / kThreads);
+    const int grid = int(tiles < 1 ? 1 : tiles < cap ? tiles : cap);
+    if (ring && !seed)
+        return launch_pdl(quantize2d_kernel<FMT, kDelayed, IN, LAYOUT>, grid, kThreads, 0, st, 1, x, rows, cols, out8,
+                          out8_t, ring, (uint32_t*)nullptr, amax_out, scale_out);
+    // current scaling or a seeded call: the flat amax pass first
+    uint32_t* acc = reinterpret_cast<uint32_t*>(amax_out);
+    const int64_t n = rows * cols;
+    if (cudaMemsetAsync(acc, 0, sizeof(uint32_t), st) != cudaSuccess) return FP8_ERR_CUDA;
+    if (launch_pdl(quantize_kernel<FMT, kAmaxOnly, IN>, grid_for(n), kThreads, 0, st, 1, x, n, (uint8_t*)nullptr,
+                   (fp8_ring*)nullptr, acc, (float*)nullptr, (float*)nullptr) != FP8_OK)
+        return FP8_ERR_CUDA;
+    if (seed)
+        return launch_pdl(quantize2d_kernel<FMT, kSeed, IN, LAYOUT>, grid, kThreads, 0, st, 1, x, rows, cols, out8,
+                          out8_t, ring, acc, (float*)nullptr, scale_out);
+    return launch_pdl(quantize2d_kernel<FMT, kCurrentQuant, IN, LAYOUT>, grid, kThreads, 0, st, 1, x, rows, cols,
+                      out8, out8_t, (fp8_ring*)nullptr, acc, (float*)nullptr, scale_out);
+}
+
+template <int FMT, int LAYOUT>
+fp8_status launch_quantize_2d_in(fp8_dtype dtype, const void* x, int64_t rows, int64_t cols, fp8_ring* ring, bool seed,
+                                 uint8_t* out8, uint8_t* out8_t, float* amax_out, float* scale_out, cudaStream_t st) {
+    switch (dtype) {
+        case FP8_IN_BF16:
+            return launch_quantize_2d<FMT, FP8_IN_BF16, LAYOUT>(x, rows, cols, ring, seed, out8, out8_t, amax_out,
+                                                                scale_out, st);
+        case FP8_IN_F16:
+            return launch_quantize_2d<FMT, FP8_IN_F16, LAYOUT>(x, rows, cols, ring, seed, out8, out8_t, amax_out,
+                                                               scale_out, st);
+        default:
+            return launch_quantize_2d<FMT, FP8_IN_F32, LAYOUT>(x, rows, cols, ring, seed, out8, out8_t, amax_out,
+                                                               scale_out, st);
+    }
+}
+
 bool scale_ok(float s) { return s > 0.0f && s <= 3.402823466e38f; }
 
 }  // namespace
@@ -442,6 +566,38 @@ extern "C" fp8_status fp8_quantize_ex(const void* x, fp8_dtype dtype, int64_t n,
     cudaStream_t st = as_stream(stream);
     return fmt == FP8_E4M3 ? launch_quantize_in<FP8_E4M3>(dtype, x, n, ring, seed, out8, amax_out, scale_out, st)
                            : launch_quantize_in<FP8_E5M2>(dtype, x, n, ring, seed, out8, amax_out, scale_out, st);
+}
+
+extern "C" fp8_status fp8_quantize_2d(const void* x, fp8_dtype dtype, int64_t rows, int64_t cols, fp8_fmt fmt,
+                                      fp8_ring* ring, uint32_t flags, fp8_quant_layout layout, uint8_t* out8,
+                                      uint8_t* out8_t, float* amax_out, float* scale_out, void* stream) {
+    if (layout != FP8_QL_ROW && layout != FP8_QL_COL && layout != FP8_QL_BOTH) return FP8_ERR_INVALID_ARG;
+    if (rows < 0 || cols < 0 || (cols > 0 && rows >= (int64_t(1) << 40) / cols)) return FP8_ERR_INVALID_ARG;
+    if (layout == FP8_QL_ROW)  // the row-major codes alone are the flat quantize
+        return fp8_quantize_ex(x, dtype, rows * cols, fmt, ring, flags, out8, amax_out, scale_out, stream);
+    if (!valid_fmt(fmt) || !valid_dtype(dtype)) return FP8_ERR_INVALID_ARG;
+    if ((flags & ~uint32_t(FP8_QUANTIZE_SEED_RING)) != 0u) return FP8_ERR_INVALID_ARG;
+    const bool seed = (flags & FP8_QUANTIZE_SEED_RING) != 0u;
+    if (seed && !ring) return FP8_ERR_INVALID_ARG;
+    if (!scale_out || ((!ring || seed) && !amax_out)) return FP8_ERR_INVALID_ARG;
+    const int64_t n = rows * cols;
+    if (n > 0 && (!x || !out8_t || (layout == FP8_QL_BOTH && !out8))) return FP8_ERR_INVALID_ARG;
+    if (rows % 8 != 0 || cols % 8 != 0) return FP8_ERR_ALIGNMENT;
+    if (!aligned(x, 16) || !aligned(out8, 16) || !aligned(out8_t, 16)) return FP8_ERR_ALIGNMENT;
+    if (ring && !aligned(ring, 4)) return FP8_ERR_ALIGNMENT;
+    if (!aligned(scale_out, 4) || !aligned(amax_out, 4)) return FP8_ERR_ALIGNMENT;
+    cudaStream_t st = as_stream(stream);
+    if (fmt == FP8_E4M3)
+        return layout == FP8_QL_COL
+                   ? launch_quantize_2d_in<FP8_E4M3, FP8_QL_COL>(dtype, x, rows, cols, ring, seed, out8, out8_t,
+                                                                 amax_out, scale_out, st)
+                   : launch_quantize_2d_in<FP8_E4M3, FP8_QL_BOTH>(dtype, x, rows, cols, ring, seed, out8, out8_t,
+                                                                  amax_out, scale_out, st);
+    return layout == FP8_QL_COL
+               ? launch_quantize_2d_in<FP8_E5M2, FP8_QL_COL>(dtype, x, rows, cols, ring, seed, out8, out8_t, amax_out,
+                                                             scale_out, st)
+               : launch_quantize_2d_in<FP8_E5M2, FP8_QL_BOTH>(dtype, x, rows, cols, ring, seed, out8, out8_t,
+                                                              amax_out, scale_out, st);
 }
 
 extern "C" fp8_status fp8_quantize(const void* x, int64_t n, fp8_fmt fmt, fp8_ring* ring, uint8_t* out8,

@@ -157,6 +157,25 @@ FP8LITE_API fp8_status fp8_quantize_ex(const void* x, fp8_dtype dtype, int64_t n
                         uint32_t flags, uint8_t* out8, float* amax_out, float* scale_out,
                         void* stream);
 
+/* Quantize of a row-major [rows, cols] tensor in either or both orientations
+ * [fp8.py@f4c44ebf, bullets on quantize(transposed) / quantize_dual and the
+ * QuantLayout enum]: the codes of x (row-major [rows, cols]), of x^T
+ * (row-major [cols, rows], i.e. the transposed copy a GEMM that wants a
+ * K-major operand reads), or both from one read of the input. Both copies
+ * hold the same bytes: out8_t[c * rows + r] == out8[r * cols + c]. The scale,
+ * amax, ring update and errors are those of fp8_quantize_ex.
+ *
+ * layout  FP8_QL_ROW: out8 only (fp8_quantize_ex on the flat tensor);
+ *         FP8_QL_COL: out8_t only; FP8_QL_BOTH: both.
+ * rows, cols  >= 0, rows * cols < 2^40; multiples of 8 when out8_t is
+ *         written (FP8_ERR_ALIGNMENT otherwise).
+ * out8    device uint8[rows * cols], 16-byte aligned (ROW, BOTH)
+ * out8_t  device uint8[cols * rows], 16-byte aligned (COL, BOTH) */
+typedef enum fp8_quant_layout { FP8_QL_ROW = 0, FP8_QL_COL = 1, FP8_QL_BOTH = 2 } fp8_quant_layout;
+FP8LITE_API fp8_status fp8_quantize_2d(const void* x, fp8_dtype dtype, int64_t rows, int64_t cols, fp8_fmt fmt,
+                        fp8_ring* ring, uint32_t flags, fp8_quant_layout layout, uint8_t* out8,
+                        uint8_t* out8_t, float* amax_out, float* scale_out, void* stream);
+
 /* Several delayed-scaling quantizations in ONE launch, e.g. the weights of
  * all layers at the start of a training step, or a layer's x and W.
  * Each job is exactly an fp8_quantize call with a ring (same arguments, same

@@ -163,3 +163,18 @@ def test_quantize_ex_validation(fp8):
     assert st(ring=None, amax=None) == fp8.FP8_ERR_INVALID_ARG           # current scaling needs amax_out
     assert st(x=A + 4, dtype=2) == fp8.FP8_ERR_ALIGNMENT                 # fp32 input still 16-byte aligned
     assert st(fmt=7) == fp8.FP8_ERR_INVALID_ARG
+
+
+def test_quantize_2d_validation(fp8):
+    def st(rows=64, cols=64, layout=2, ring=S, flags=0, out8=A + 4096, out8_t=A + 8192, dtype=0, amax=S + 128):
+        return fp8.raw_status("fp8_quantize_2d", A, dtype, rows, cols, 0, ring, flags, layout, out8, out8_t, amax,
+                              S + 64, None)
+    assert st(layout=3) == fp8.FP8_ERR_INVALID_ARG
+    assert st(rows=-8) == fp8.FP8_ERR_INVALID_ARG
+    assert st(rows=60) == fp8.FP8_ERR_ALIGNMENT            # the transposed copy needs multiples of 8
+    assert st(cols=12) == fp8.FP8_ERR_ALIGNMENT
+    assert st(out8_t=None) == fp8.FP8_ERR_INVALID_ARG
+    assert st(layout=2, out8=None) == fp8.FP8_ERR_INVALID_ARG
+    assert st(layout=1, out8=None, out8_t=A + 8200) == fp8.FP8_ERR_ALIGNMENT
+    assert st(ring=None, flags=1) == fp8.FP8_ERR_INVALID_ARG
+    assert st(dtype=5) == fp8.FP8_ERR_INVALID_ARG

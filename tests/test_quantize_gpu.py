@@ -327,3 +327,80 @@ def test_seeded_first_call(g, dtype):
         hist, rs, idx, acc, ticket = g.ring_state(ring)
         assert np.array_equal(hist, ref.hist) and rs == ref.scale and idx == ref.idx, step
         assert acc == 0 and ticket == 0
+
+
+# ------------------------------------------------ transposed / dual codes ---
+
+def _q2d(g, x, dtype, rows, cols, fmt, ring, flags, layout):
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    n = rows * cols
+    out = torch.full((max(n, 16),), 0xAB, dtype=torch.uint8, device="cuda")
+    out_t = torch.full((max(n, 16),), 0xCD, dtype=torch.uint8, device="cuda")
+    amax = torch.full((1,), -1.0, device="cuda")
+    scale = torch.full((1,), -1.0, device="cuda")
+    fp8.fp8_quantize_2d(x, dtype, rows, cols, fmt, ring, flags, layout, out, out_t, amax, scale)
+    return out[:n], out_t[:n], amax, scale
+
+
+@pytest.mark.parametrize("rows,cols", [(64, 64), (8, 8), (200, 136), (1024, 2056), (4096, 1024), (8, 4104)])
+@pytest.mark.parametrize("dtype", [0, 1, 2])
+def test_dual_quantize_byte_equality_and_oracle(g, rows, cols, dtype):
+    """Both orientations from one pass hold the same bytes, the row-major copy
+    is the oracle's codes, and the ring moves as for the flat quantize."""
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    torch_dt = {0: torch.bfloat16, 1: torch.float16, 2: torch.float32}[dtype]
+    ring = g.new_ring()
+    ref = oracle.DelayedRing()
+    for step in range(3):
+        x = (W.bf16_normal((rows, cols), 0.05, 9500 + rows + step).float() * (1 + step)).to(torch_dt)
+        xd = x.cuda()
+        out, out_t, amax, scale = _q2d(g, xd, dtype, rows, cols, E4M3, ring, 0, fp8.FP8_QL_BOTH)
+        want, a, s = ref.step(x.float().numpy().reshape(-1), E4M3)
+        got = g.codes(out)
+        assert np.array_equal(got, want), step
+        assert np.array_equal(g.codes(out_t).reshape(cols, rows), got.reshape(rows, cols).T), step
+        assert g.f32(scale)[0] == s and g.f32(amax)[0] == a
+        hist, rs, idx, acc, ticket = g.ring_state(ring)
+        assert np.array_equal(hist, ref.hist) and rs == ref.scale and idx == ref.idx and acc == 0 and ticket == 0
+    # the transposed copy alone: the same bytes, and the row-major buffer untouched
+    ring2 = g.new_ring()
+    ring2_ref = oracle.DelayedRing()
+    out, out_t, _, scale = _q2d(g, xd, dtype, rows, cols, E4M3, ring2, 0, fp8.FP8_QL_COL)
+    want, _, s = ring2_ref.step(x.float().numpy().reshape(-1), E4M3)
+    assert np.array_equal(g.codes(out_t).reshape(cols, rows), want.reshape(rows, cols).T)
+    assert (g.codes(out) == 0xAB).all() and g.f32(scale)[0] == s
+
+
+@pytest.mark.parametrize("flags", [0, 1])
+def test_dual_quantize_current_and_seeded(g, flags):
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    rows, cols = 512, 776
+    x = W.f32_mixed(rows * cols, 9600 + flags)
+    x[~torch.isfinite(x)] = 0.0
+    x = x.reshape(rows, cols)
+    ring = g.new_ring() if flags else None
+    out, out_t, amax, scale = _q2d(g, x.cuda(), fp8.FP8_IN_F32, rows, cols, E5M2, ring, flags, fp8.FP8_QL_BOTH)
+    if flags:
+        ref = oracle.DelayedRing()
+        want, a, s = ref.seed_step(x.numpy().reshape(-1), E5M2)
+        hist, rs, idx, _, _ = g.ring_state(ring)
+        assert np.array_equal(hist, ref.hist) and rs == ref.scale and idx == ref.idx
+    else:
+        want, a, s = oracle.quantize_current(x.numpy().reshape(-1), E5M2)
+    got = g.codes(out)
+    assert np.array_equal(got, want)
+    assert np.array_equal(g.codes(out_t).reshape(cols, rows), got.reshape(rows, cols).T)
+    assert g.f32(amax)[0] == a and g.f32(scale)[0] == s
+
+
+def test_dual_quantize_empty_and_row_layout(g):
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    ring = g.new_ring(2.0)
+    out, out_t, amax, scale = _q2d(g, None, 0, 0, 64, E4M3, ring, 0, fp8.FP8_QL_BOTH)
+    hist, rs, idx, _, _ = g.ring_state(ring)
+    assert idx == 1 and rs == np.float32(2.0) and g.f32(scale)[0] == np.float32(2.0)
+    # FP8_QL_ROW is the flat quantize
+    x = W.bf16_normal((96, 40), 1.0, 9700).cuda()
+    out, _, _, _ = _q2d(g, x, 0, 96, 40, E4M3, None, 0, fp8.FP8_QL_ROW)
+    want, _, _ = oracle.quantize_current(x.float().cpu().numpy().reshape(-1), E4M3)
+    assert np.array_equal(g.codes(out), want)
