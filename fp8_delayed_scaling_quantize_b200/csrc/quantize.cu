@@ -291,70 +291,90 @@ quantize_kernel(const void* __restrict__ x, int64_t n, uint8_t* __restrict__ out
 
 // Quantize of a [rows, cols] tensor that also writes the transposed codes
 // [cols, rows] (LAYOUT FP8_QL_COL: only those; FP8_QL_BOTH: both, from one read
-// of the input). A block walks 64 x 64 tiles: each thread quantizes one 8-element
-// unit of a row (exactly as the flat kernel does, so both orientations hold
-// the same bytes), writes it to the row-major codes, and drops its 8 codes into a
-// shared-memory tile column; after a barrier each thread reads 8 consecutive
-// codes of a tile row, which are 8 consecutive rows of one input column, and
-// writes them to the transposed codes. rows and cols are multiples of 8.
-constexpr int kTile = 64;
-constexpr int kTileStride = kTile + 4;  // bytes per shared tile row: 4-byte reads, 2-way conflicts on the writes
+// of the input). A block walks 128 x 64 tiles (rows x columns): each thread
+// quantizes two 8-element units of a row (rows lr and lr + 64, exactly as the
+// flat kernel does, so both orientations hold the same bytes), writes them to
+// the row-major codes, and drops their codes into a shared-memory tile held
+// column-major; after a barrier each thread reads 16 consecutive codes of one
+// tile column (16 consecutive rows of one input column) and writes them to the
+// transposed codes. The next tile's loads leave before the current tile is
+// processed. rows and cols are multiples of 8.
+constexpr int kTileR = 128, kTileC = 64;
+constexpr int kTileStride = kTileR + 4;  // bytes per shared tile column: 4-byte reads, 2-way conflicts on the writes
+
+template <int IN>
+__device__ __forceinline__ void load_tile_units(const void* x, int64_t rows, int64_t cols, int64_t r0, int64_t c0,
+                                                int lr, int lc, Unit (&v)[2], bool (&have)[2]) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int64_t r = r0 + lr + h * (kTileR / 2);
+        have[h] = r < rows && c0 + lc < cols;
+        if (have[h]) load_unit<IN>(x, (r * cols + c0 + lc) >> 3, v[h]);
+    }
+}
 
 template <int FMT, int MODE, int IN, int LAYOUT>
 __global__ void __launch_bounds__(kThreads)
 quantize2d_kernel(const void* __restrict__ x, int64_t rows, int64_t cols, uint8_t* __restrict__ out8,
                   uint8_t* __restrict__ out8_t, fp8_ring* ring, uint32_t* amax_acc, float* amax_out,
                   float* scale_out) {
-    static_assert(kThreads == kTile * kTile / 8, "one unit per thread and tile");
+    static_assert(kThreads * 16 == kTileR * kTileC, "two units per thread and tile");
     __shared__ float s_scale;
-    __shared__ __align__(16) uint8_t tile[kTile][kTileStride];
+    __shared__ __align__(16) uint8_t tile[kTileC][kTileStride];
     griddep_wait();
-    const int64_t trows = (rows + kTile - 1) / kTile, tcols = (cols + kTile - 1) / kTile;
-    const int64_t tiles = trows * tcols;
-    const int lr = threadIdx.x >> 3;        // tile row this thread loads
-    const int lc = (threadIdx.x & 7) * 8;   // its first tile column
-    const int oc = threadIdx.x >> 3;        // tile column (transposed row) it writes
-    const int orow = (threadIdx.x & 7) * 8; // its first tile row there
-    // the first tile's load leaves before the scale is known
+    const int64_t tcols = (cols + kTileC - 1) / kTileC;
+    const int64_t tiles = ((rows + kTileR - 1) / kTileR) * tcols;
+    const int lr = threadIdx.x >> 3;         // tile rows lr and lr + 64 this thread loads
+    const int lc = (threadIdx.x & 7) * 8;    // its first tile column
+    const int oc = threadIdx.x >> 3;         // tile column (transposed row) it writes
+    const int orow = (threadIdx.x & 7) * 16; // its first tile row there
+    // the first tile's loads leave before the scale is known
     int64_t t = blockIdx.x;
-    Unit v;
+    Unit v[2];
+    bool have[2] = {false, false};
     int64_t r0 = 0, c0 = 0;
-    bool have = false;
     if (t < tiles) {
-        r0 = (t / tcols) * kTile;
-        c0 = (t % tcols) * kTile;
-        have = r0 + lr < rows && c0 + lc < cols;
-        if (have) load_unit<IN>(x, ((r0 + lr) * cols + c0 + lc) >> 3, v);
+        r0 = (t / tcols) * kTileR;
+        c0 = (t % tcols) * kTileC;
+        load_tile_units<IN>(x, rows, cols, r0, c0, lr, lc, v, have);
     }
     const float s = read_scale<FMT, MODE>(ring, amax_acc, scale_out, blockIdx.x, s_scale);
     float m = 0.0f;
     while (t < tiles) {
-        uint2 q = make_uint2(0u, 0u);
-        if (have) {
-            float f[8];
-            unit_f32<IN>(v, f);
-            q = quant8<FMT>(f, s, m);
-            if (LAYOUT == FP8_QL_BOTH) *reinterpret_cast<uint2*>(out8 + (r0 + lr) * cols + c0 + lc) = q;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            uint2 q = make_uint2(0u, 0u);
+            const int r = lr + h * (kTileR / 2);
+            if (have[h]) {
+                float f[8];
+                unit_f32<IN>(v[h], f);
+                q = quant8<FMT>(f, s, m);
+                if (LAYOUT == FP8_QL_BOTH) *reinterpret_cast<uint2*>(out8 + (r0 + r) * cols + c0 + lc) = q;
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                tile[lc + k][r] = uint8_t(q.x >> (8 * k));
+                tile[lc + 4 + k][r] = uint8_t(q.y >> (8 * k));
+            }
+        }
+        __syncthreads();
+        const int64_t tr0 = r0, tc0 = c0;
+        t += gridDim.x;
+        if (t < tiles) {  // the next tile's loads, in flight while this one is written out
+            r0 = (t / tcols) * kTileR;
+            c0 = (t % tcols) * kTileC;
+            load_tile_units<IN>(x, rows, cols, r0, c0, lr, lc, v, have);
         }
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            tile[lc + k][lr] = uint8_t(q.x >> (8 * k));
-            tile[lc + 4 + k][lr] = uint8_t(q.y >> (8 * k));
+        for (int g8 = 0; g8 < 2; ++g8) {  // two groups of 8 rows (rows is a multiple of 8)
+            const int rr = orow + 8 * g8;
+            if (tc0 + oc < cols && tr0 + rr < rows) {
+                const uint32_t w0 = *reinterpret_cast<const uint32_t*>(&tile[oc][rr]);
+                const uint32_t w1 = *reinterpret_cast<const uint32_t*>(&tile[oc][rr + 4]);
+                *reinterpret_cast<uint2*>(out8_t + (tc0 + oc) * rows + tr0 + rr) = make_uint2(w0, w1);
+            }
         }
-        __syncthreads();
-        if (c0 + oc < cols && r0 + orow < rows) {
-            const uint32_t w0 = *reinterpret_cast<const uint32_t*>(&tile[oc][orow]);
-            const uint32_t w1 = *reinterpret_cast<const uint32_t*>(&tile[oc][orow + 4]);
-            *reinterpret_cast<uint2*>(out8_t + (c0 + oc) * rows + r0 + orow) = make_uint2(w0, w1);
-        }
-        t += gridDim.x;
-        if (t < tiles) {  // the next tile's load, then the barrier that frees the shared tile
-            r0 = (t / tcols) * kTile;
-            c0 = (t % tcols) * kTile;
-            have = r0 + lr < rows && c0 + lc < cols;
-            if (have) load_unit<IN>(x, ((r0 + lr) * cols + c0 + lc) >> 3, v);
-        }
-        __syncthreads();
+        __syncthreads();  // the shared tile is free for the next tile
     }
     griddep_launch();
     finish_block<FMT, MODE>(m, ring, amax_acc, amax_out, blockIdx.x, gridDim.x);
@@ -465,7 +485,7 @@ bool valid_dtype(int d) { return d == FP8_IN_BF16 || d == FP8_IN_F16 || d == FP8
 template <int FMT, int IN, int LAYOUT>
 fp8_status launch_quantize_2d(const void* x, int64_t rows, int64_t cols, fp8_ring* ring, bool seed, uint8_t* out8,
                               uint8_t* out8_t, float* amax_out, float* scale_out, cudaStream_t st) {
-    const int64_t tiles = ((rows + kTile - 1) / kTile) * ((cols + kTile - 1) / kTile);
+    const int64_t tiles = ((rows + kTileR - 1) / kTileR) * ((cols + kTileC - 1) / kTileC);
     const int64_t cap = int64_t(sm_count()) * (2048 / kThreads);
     const int grid = int(tiles < 1 ? 1 : tiles < cap ? tiles : cap);
     if (ring && !seed)
