@@ -28,6 +28,7 @@ FP8_RING_BYTES = 80
 FP8_IN_BF16, FP8_IN_F16, FP8_IN_F32 = 0, 1, 2
 FP8_QL_ROW, FP8_QL_COL, FP8_QL_BOTH = 0, 1, 2
 FP8_QUANTIZE_SEED_RING = 1
+FP8_QUANTIZE_DEFER_FOLD = 2
 
 
 class Fp8Error(RuntimeError):
@@ -76,6 +77,8 @@ def _load():
         "fp8_selftest_wait_timeout": (I, [ctypes.c_uint32, P]),
         "fp8_bias_grad": (I, [P, I64, I64, P, P]),
         "fp8_quantize_many": (I, [P, ctypes.c_int32, P]),
+        "fp8_quantize_many_ex": (I, [P, ctypes.c_int32, ctypes.c_uint32, P]),
+        "fp8_rings_fold": (I, [P, ctypes.c_int32, P, P]),
         "fp8_mm_ws": (I, [P, I, P, I, P, P, I, I64, I64, I64, I64, I64, I64, I64, P, P, I, P, P, ctypes.c_size_t,
                           ctypes.c_int32, P]),
         "fp8_mm_workspace_size": (ctypes.c_size_t, [I64, I64, I64, I64, I, ctypes.c_int32]),
@@ -158,7 +161,14 @@ def fp8_quantize_2d(x, dtype, rows, cols, fmt, ring, flags, layout, out8, out8_t
                                       _stream(stream)), "fp8_quantize_2d")
 
 
-def fp8_quantize_many(jobs, stream=None):
+def fp8_rings_fold(rings, count, fmts, stream=None):
+    """Fold the accumulated amax of `count` consecutive rings; fmts: ints."""
+    arr = (ctypes.c_int32 * max(len(fmts), 1))(*[int(f) for f in fmts])
+    return _check(lib.fp8_rings_fold(_ptr(rings), int(count), ctypes.cast(arr, ctypes.c_void_p), _stream(stream)),
+                  "fp8_rings_fold")
+
+
+def fp8_quantize_many(jobs, stream=None, flags=0):
     """jobs: sequence of (x, n, fmt, ring, out8, amax_out, scale_out[, dtype])."""
     arr = (fp8_quantize_job * max(len(jobs), 1))()
     for i, job in enumerate(jobs):
@@ -166,8 +176,8 @@ def fp8_quantize_many(jobs, stream=None):
         dtype = job[7] if len(job) > 7 else FP8_IN_BF16
         arr[i] = fp8_quantize_job(_ptr(x), int(n), int(fmt), int(dtype), _ptr(ring), _ptr(out8), _ptr(amax_out),
                                   _ptr(scale_out))
-    return _check(lib.fp8_quantize_many(ctypes.cast(arr, ctypes.c_void_p), len(jobs), _stream(stream)),
-                  "fp8_quantize_many")
+    return _check(lib.fp8_quantize_many_ex(ctypes.cast(arr, ctypes.c_void_p), len(jobs), int(flags),
+                                           _stream(stream)), "fp8_quantize_many")
 
 
 def fp8_mm(a8, fa, b8, fb, sa, sb, layout, M, N, K, batch, stride_a, stride_b, stride_c, bias,

@@ -45,7 +45,9 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kUnroll = 4;  // 16-byte units in flight per thread
 
-enum Mode { kDelayed = 0, kCurrentQuant = 1, kAmaxOnly = 2, kSeed = 3 };
+// kDeferred: a delayed call whose fold is left to fp8_rings_fold, so that the
+// ranks of a data-parallel group can first all-reduce the ring's amax.
+enum Mode { kDelayed = 0, kCurrentQuant = 1, kAmaxOnly = 2, kSeed = 3, kDeferred = 4 };
 
 template <int FMT>
 __device__ __forceinline__ uint32_t cvt_pair(float lo, float hi) {
@@ -164,17 +166,23 @@ __device__ __forceinline__ void finish_block(float m, fp8_ring* ring, uint32_t* 
     if (MODE == kSeed) {
         if (blk != 0 || threadIdx.x != 0) return;  // block 0 folds the amax into the ring
     } else {
+        constexpr bool kRing = MODE == kDelayed || MODE == kDeferred;
         const uint32_t bits = block_max_bits(m);
         if (threadIdx.x != 0) return;
-        uint32_t* acc = MODE == kDelayed ? &ring->amax_bits : amax_acc;
+        uint32_t* acc = kRing ? &ring->amax_bits : amax_acc;
         if (bits != 0u) atomicMax(acc, bits);
-        if (MODE != kDelayed) return;
+        if (!kRing) return;
         // Last-block election: every block publishes its amax, then takes a
         // ticket with acquire-release semantics (its amax is visible before
         // the ticket moves); the block holding the final ticket sees every
         // amax.
         const uint32_t ticket = atom_add_acq_rel(&ring->ticket, 1u);
         if (ticket != uint32_t(nblk) - 1) return;
+        if (MODE == kDeferred) {  // the accumulator keeps this call's amax for the exchange and the fold
+            if (amax_out) *amax_out = __uint_as_float(*reinterpret_cast<volatile uint32_t*>(&ring->amax_bits));
+            reinterpret_cast<volatile fp8_ring*>(ring)->ticket = 0u;
+            return;
+        }
     }
     // The history and its index change only in this finalize, so they are
     // read together with the exchange of the accumulated amax: the 18
@@ -209,7 +217,7 @@ __device__ __forceinline__ float read_scale(fp8_ring* ring, uint32_t* amax_acc, 
                                             float& s_scale) {
     if (threadIdx.x == 0) {
         float v;
-        if (MODE == kDelayed) {
+        if (MODE == kDelayed || MODE == kDeferred) {
             v = *reinterpret_cast<volatile float*>(&ring->scale);
         } else {  // current scaling, also the seeded call: from the measured amax
             const float a = __uint_as_float(*reinterpret_cast<volatile uint32_t*>(amax_acc));
@@ -397,6 +405,7 @@ struct QuantJobs {
     float* scale_out[FP8_QUANTIZE_MAX_JOBS];
 };
 
+template <int MODE>
 __global__ void __launch_bounds__(kThreads) quantize_many_kernel(const __grid_constant__ QuantJobs jobs) {
     __shared__ float s_scale;
     griddep_wait();
@@ -404,7 +413,7 @@ __global__ void __launch_bounds__(kThreads) quantize_many_kernel(const __grid_co
     while (j + 1 < jobs.count && int(blockIdx.x) >= jobs.first[j + 1]) ++j;
     const int blk = int(blockIdx.x) - jobs.first[j];
 #define FP8LITE_JOB(F, I)                                                                                        \
-    quantize_body<F, kDelayed, I>(jobs.x[j], jobs.n[j], jobs.out8[j], jobs.ring[j], nullptr, jobs.amax_out[j], \
+    quantize_body<F, MODE, I>(jobs.x[j], jobs.n[j], jobs.out8[j], jobs.ring[j], nullptr, jobs.amax_out[j],     \
                                   jobs.scale_out[j], blk, jobs.blocks[j], s_scale)
     const int dt = jobs.dtype[j];
     if (jobs.fmt[j] == FP8_E4M3) {
@@ -431,6 +440,32 @@ __global__ void ring_write_kernel(fp8_ring* ring, fp8_ring value) {
     }
 }
 
+// Folds each ring's accumulated amax (a deferred call's, after the group's
+// all-reduce) into its history exactly as a delayed call's last block does.
+constexpr int kMaxFoldRings = 64;
+struct FoldFmts {
+    int fmt[kMaxFoldRings];
+};
+
+__global__ void rings_fold_kernel(fp8_ring* rings, int count, const __grid_constant__ FoldFmts f) {
+    griddep_wait();
+    const int i = threadIdx.x;
+    if (i < count) {
+        volatile fp8_ring* r = rings + i;
+        const float a = __uint_as_float(r->amax_bits);
+        const uint32_t idx = r->idx & (FP8_RING_HISTORY - 1);
+        float wmax = a;
+#pragma unroll
+        for (int k = 0; k < FP8_RING_HISTORY; ++k)
+            if (uint32_t(k) != idx) wmax = fmaxf(wmax, r->hist[k]);
+        r->hist[idx] = a;
+        if (wmax > 0.0f && isfinite(wmax)) r->scale = scale_from_amax(fmt_max(f.fmt[i]), wmax);
+        r->idx = (idx + 1) & (FP8_RING_HISTORY - 1);
+        r->amax_bits = 0u;
+    }
+    griddep_launch();
+}
+
 int sm_count() {
     static int cached[64] = {0};
     int dev = 0;
@@ -452,9 +487,12 @@ int grid_for(int64_t n) {
 }
 
 template <int FMT, int IN>
-fp8_status launch_quantize(const void* x, int64_t n, fp8_ring* ring, bool seed, uint8_t* out8, float* amax_out,
-                           float* scale_out, cudaStream_t st) {
+fp8_status launch_quantize(const void* x, int64_t n, fp8_ring* ring, bool seed, bool defer, uint8_t* out8,
+                           float* amax_out, float* scale_out, cudaStream_t st) {
     const int grid = grid_for(n);
+    if (ring && defer)
+        return launch_pdl(quantize_kernel<FMT, kDeferred, IN>, grid, kThreads, 0, st, 1, x, n, out8, ring,
+                          (uint32_t*)nullptr, amax_out, scale_out);
     if (ring && !seed)
         return launch_pdl(quantize_kernel<FMT, kDelayed, IN>, grid, kThreads, 0, st, 1, x, n, out8, ring,
                           (uint32_t*)nullptr, amax_out, scale_out);
@@ -471,12 +509,15 @@ fp8_status launch_quantize(const void* x, int64_t n, fp8_ring* ring, bool seed, 
 }
 
 template <int FMT>
-fp8_status launch_quantize_in(fp8_dtype dtype, const void* x, int64_t n, fp8_ring* ring, bool seed, uint8_t* out8,
-                              float* amax_out, float* scale_out, cudaStream_t st) {
+fp8_status launch_quantize_in(fp8_dtype dtype, const void* x, int64_t n, fp8_ring* ring, bool seed, bool defer,
+                              uint8_t* out8, float* amax_out, float* scale_out, cudaStream_t st) {
     switch (dtype) {
-        case FP8_IN_BF16: return launch_quantize<FMT, FP8_IN_BF16>(x, n, ring, seed, out8, amax_out, scale_out, st);
-        case FP8_IN_F16:  return launch_quantize<FMT, FP8_IN_F16>(x, n, ring, seed, out8, amax_out, scale_out, st);
-        default:          return launch_quantize<FMT, FP8_IN_F32>(x, n, ring, seed, out8, amax_out, scale_out, st);
+        case FP8_IN_BF16:
+            return launch_quantize<FMT, FP8_IN_BF16>(x, n, ring, seed, defer, out8, amax_out, scale_out, st);
+        case FP8_IN_F16:
+            return launch_quantize<FMT, FP8_IN_F16>(x, n, ring, seed, defer, out8, amax_out, scale_out, st);
+        default:
+            return launch_quantize<FMT, FP8_IN_F32>(x, n, ring, seed, defer, out8, amax_out, scale_out, st);
     }
 }
 
@@ -573,9 +614,11 @@ extern "C" fp8_status fp8_quantize_ex(const void* x, fp8_dtype dtype, int64_t n,
                                       uint32_t flags, uint8_t* out8, float* amax_out, float* scale_out,
                                       void* stream) {
     if (!valid_fmt(fmt) || !valid_dtype(dtype)) return FP8_ERR_INVALID_ARG;
-    if ((flags & ~uint32_t(FP8_QUANTIZE_SEED_RING)) != 0u) return FP8_ERR_INVALID_ARG;
+    if ((flags & ~uint32_t(FP8_QUANTIZE_SEED_RING | FP8_QUANTIZE_DEFER_FOLD)) != 0u) return FP8_ERR_INVALID_ARG;
     const bool seed = (flags & FP8_QUANTIZE_SEED_RING) != 0u;
-    if (seed && !ring) return FP8_ERR_INVALID_ARG;
+    const bool defer = (flags & FP8_QUANTIZE_DEFER_FOLD) != 0u;
+    if ((seed || defer) && !ring) return FP8_ERR_INVALID_ARG;
+    if (seed && defer) return FP8_ERR_INVALID_ARG;
     if (n < 0 || n >= (int64_t(1) << 40)) return FP8_ERR_INVALID_ARG;
     if (!scale_out) return FP8_ERR_INVALID_ARG;
     if (n > 0 && (!x || !out8)) return FP8_ERR_INVALID_ARG;
@@ -584,8 +627,9 @@ extern "C" fp8_status fp8_quantize_ex(const void* x, fp8_dtype dtype, int64_t n,
     if (ring && !aligned(ring, 4)) return FP8_ERR_ALIGNMENT;
     if (!aligned(scale_out, 4) || !aligned(amax_out, 4)) return FP8_ERR_ALIGNMENT;
     cudaStream_t st = as_stream(stream);
-    return fmt == FP8_E4M3 ? launch_quantize_in<FP8_E4M3>(dtype, x, n, ring, seed, out8, amax_out, scale_out, st)
-                           : launch_quantize_in<FP8_E5M2>(dtype, x, n, ring, seed, out8, amax_out, scale_out, st);
+    return fmt == FP8_E4M3
+               ? launch_quantize_in<FP8_E4M3>(dtype, x, n, ring, seed, defer, out8, amax_out, scale_out, st)
+               : launch_quantize_in<FP8_E5M2>(dtype, x, n, ring, seed, defer, out8, amax_out, scale_out, st);
 }
 
 extern "C" fp8_status fp8_quantize_2d(const void* x, fp8_dtype dtype, int64_t rows, int64_t cols, fp8_fmt fmt,
@@ -593,6 +637,7 @@ extern "C" fp8_status fp8_quantize_2d(const void* x, fp8_dtype dtype, int64_t ro
                                       uint8_t* out8_t, float* amax_out, float* scale_out, void* stream) {
     if (layout != FP8_QL_ROW && layout != FP8_QL_COL && layout != FP8_QL_BOTH) return FP8_ERR_INVALID_ARG;
     if (rows < 0 || cols < 0 || (cols > 0 && rows >= (int64_t(1) << 40) / cols)) return FP8_ERR_INVALID_ARG;
+    if (flags & FP8_QUANTIZE_DEFER_FOLD) return FP8_ERR_INVALID_ARG;  // offered by the flat quantize only
     if (layout == FP8_QL_ROW)  // the row-major codes alone are the flat quantize
         return fp8_quantize_ex(x, dtype, rows * cols, fmt, ring, flags, out8, amax_out, scale_out, stream);
     if (!valid_fmt(fmt) || !valid_dtype(dtype)) return FP8_ERR_INVALID_ARG;
@@ -620,13 +665,26 @@ extern "C" fp8_status fp8_quantize_2d(const void* x, fp8_dtype dtype, int64_t ro
                                                               amax_out, scale_out, st);
 }
 
+extern "C" fp8_status fp8_rings_fold(fp8_ring* rings, int32_t count, const int32_t* fmts, void* stream) {
+    if (!rings || !fmts || count < 1 || count > kMaxFoldRings) return FP8_ERR_INVALID_ARG;
+    if (!aligned(rings, 4)) return FP8_ERR_ALIGNMENT;
+    FoldFmts f = {};
+    for (int i = 0; i < count; ++i) {
+        if (!valid_fmt(fmts[i])) return FP8_ERR_INVALID_ARG;
+        f.fmt[i] = fmts[i];
+    }
+    return launch_pdl(rings_fold_kernel, 1, kMaxFoldRings, 0, as_stream(stream), 1, rings, int(count), f);
+}
+
 extern "C" fp8_status fp8_quantize(const void* x, int64_t n, fp8_fmt fmt, fp8_ring* ring, uint8_t* out8,
                                    float* amax_out, float* scale_out, void* stream) {
     return fp8_quantize_ex(x, FP8_IN_BF16, n, fmt, ring, 0u, out8, amax_out, scale_out, stream);
 }
 
-extern "C" fp8_status fp8_quantize_many(const fp8_quantize_job* jobs, int32_t count, void* stream) {
+extern "C" fp8_status fp8_quantize_many_ex(const fp8_quantize_job* jobs, int32_t count, uint32_t flags,
+                                           void* stream) {
     if (!jobs || count < 1 || count > FP8_QUANTIZE_MAX_JOBS) return FP8_ERR_INVALID_ARG;
+    if ((flags & ~uint32_t(FP8_QUANTIZE_DEFER_FOLD)) != 0u) return FP8_ERR_INVALID_ARG;
     QuantJobs q = {};
     q.count = count;
     int total = 0;
@@ -652,5 +710,11 @@ extern "C" fp8_status fp8_quantize_many(const fp8_quantize_job* jobs, int32_t co
         q.amax_out[j] = in.amax_out;
         q.scale_out[j] = in.scale_out;
     }
-    return launch_pdl(quantize_many_kernel, total, kThreads, 0, as_stream(stream), 1, q);
+    if (flags & FP8_QUANTIZE_DEFER_FOLD)
+        return launch_pdl(quantize_many_kernel<kDeferred>, total, kThreads, 0, as_stream(stream), 1, q);
+    return launch_pdl(quantize_many_kernel<kDelayed>, total, kThreads, 0, as_stream(stream), 1, q);
+}
+
+extern "C" fp8_status fp8_quantize_many(const fp8_quantize_job* jobs, int32_t count, void* stream) {
+    return fp8_quantize_many_ex(jobs, count, 0u, stream);
 }

@@ -149,13 +149,34 @@ FP8LITE_API fp8_status fp8_quantize(const void* x, int64_t n, fp8_fmt fmt, fp8_r
  *        (a memset and two launches); amax_out is then REQUIRED (it is the
  *        accumulator).
  * Other arguments, results and errors as fp8_quantize (x 16-byte aligned
- * whatever its type); FP8_ERR_INVALID_ARG also for an unknown dtype or flag
- * and for FP8_QUANTIZE_SEED_RING without a ring. */
+ * whatever its type); FP8_ERR_INVALID_ARG also for an unknown dtype or flag,
+ * for FP8_QUANTIZE_SEED_RING or FP8_QUANTIZE_DEFER_FOLD without a ring, and
+ * for both flags together. */
 typedef enum fp8_dtype { FP8_IN_BF16 = 0, FP8_IN_F16 = 1, FP8_IN_F32 = 2 } fp8_dtype;
 #define FP8_QUANTIZE_SEED_RING 1u
+/* FP8_QUANTIZE_DEFER_FOLD (with a ring, not with SEED): a delayed call that
+ * quantizes with ring->scale and leaves this call's amax in the ring's
+ * accumulator (amax_bits, as fp32 bits) instead of folding it: the ranks of
+ * a data-parallel group all-reduce those 4 bytes with MAX (non-negative fp32
+ * bit patterns order like unsigned integers) and then call fp8_rings_fold, so
+ * every replica's ring sees the group's amax and stays identical. amax_out
+ * (optional) receives this rank's own amax. Until the fold the ring must not
+ * be used by another call. */
+#define FP8_QUANTIZE_DEFER_FOLD 2u
 FP8LITE_API fp8_status fp8_quantize_ex(const void* x, fp8_dtype dtype, int64_t n, fp8_fmt fmt, fp8_ring* ring,
                         uint32_t flags, uint8_t* out8, float* amax_out, float* scale_out,
                         void* stream);
+
+/* Folds the amax accumulated in each of `count` rings (by deferred calls, and
+ * all-reduced over a data-parallel group) into its history: hist[idx] = amax,
+ * idx + 1, the window's max publishes the next scale (as the last block of a
+ * delayed call does), the accumulator is reset. One launch for all rings.
+ * rings   device array of `count` consecutive rings (e.g. a layer's x, W and g)
+ * count   1 .. 64
+ * fmts    host int32[count]: each ring's fp8_fmt (its fmt_max sets the scale)
+ * Errors: FP8_ERR_INVALID_ARG (count, NULL, bad fmt), FP8_ERR_ALIGNMENT,
+ *         FP8_ERR_CUDA. */
+FP8LITE_API fp8_status fp8_rings_fold(fp8_ring* rings, int32_t count, const int32_t* fmts, void* stream);
 
 /* Quantize of a row-major [rows, cols] tensor in either or both orientations
  * [fp8.py@f4c44ebf, bullets on quantize(transposed) / quantize_dual and the
@@ -196,6 +217,11 @@ typedef struct fp8_quantize_job {
     float* scale_out;  /* required: the scale this job used */
 } fp8_quantize_job;
 FP8LITE_API fp8_status fp8_quantize_many(const fp8_quantize_job* jobs, int32_t count, void* stream);
+/* fp8_quantize_many with flags: 0, or FP8_QUANTIZE_DEFER_FOLD for every job
+ * (each job's amax stays in its ring's accumulator for a data-parallel
+ * all-reduce and fp8_rings_fold; see fp8_quantize_ex). */
+FP8LITE_API fp8_status fp8_quantize_many_ex(const fp8_quantize_job* jobs, int32_t count, uint32_t flags,
+                                            void* stream);
 
 /* Per-tensor-scaled FP8 GEMM with fused bias and bf16 output
  * [fp8.py@f4c44ebf, bullets on the fused bias and 3-D operands;

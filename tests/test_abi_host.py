@@ -157,7 +157,9 @@ def test_quantize_ex_validation(fp8):
         return fp8.raw_status("fp8_quantize_ex", x, dtype, n, fmt, ring, flags, out8, amax, scale, None)
     assert st(dtype=3) == fp8.FP8_ERR_INVALID_ARG
     assert st(dtype=-1) == fp8.FP8_ERR_INVALID_ARG
-    assert st(flags=2) == fp8.FP8_ERR_INVALID_ARG                        # unknown flag
+    assert st(flags=4) == fp8.FP8_ERR_INVALID_ARG                        # unknown flag
+    assert st(flags=3) == fp8.FP8_ERR_INVALID_ARG                        # seed and deferred fold together
+    assert st(ring=None, flags=fp8.FP8_QUANTIZE_DEFER_FOLD, amax=S + 128) == fp8.FP8_ERR_INVALID_ARG
     assert st(ring=None, flags=fp8.FP8_QUANTIZE_SEED_RING) == fp8.FP8_ERR_INVALID_ARG  # seed needs a ring
     assert st(flags=fp8.FP8_QUANTIZE_SEED_RING, amax=None) == fp8.FP8_ERR_INVALID_ARG  # seed needs amax_out
     assert st(ring=None, amax=None) == fp8.FP8_ERR_INVALID_ARG           # current scaling needs amax_out
@@ -178,3 +180,18 @@ def test_quantize_2d_validation(fp8):
     assert st(layout=1, out8=None, out8_t=A + 8200) == fp8.FP8_ERR_ALIGNMENT
     assert st(ring=None, flags=1) == fp8.FP8_ERR_INVALID_ARG
     assert st(dtype=5) == fp8.FP8_ERR_INVALID_ARG
+
+
+def test_rings_fold_and_grouped_flags_validation(fmt_ok=(0, 1)):
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    arr = (ctypes.c_int32 * 3)(0, 1, 0)
+    assert fp8.raw_status("fp8_rings_fold", None, 3, ctypes.cast(arr, ctypes.c_void_p), None) == fp8.FP8_ERR_INVALID_ARG
+    assert fp8.raw_status("fp8_rings_fold", S, 0, ctypes.cast(arr, ctypes.c_void_p), None) == fp8.FP8_ERR_INVALID_ARG
+    assert fp8.raw_status("fp8_rings_fold", S, 65, ctypes.cast(arr, ctypes.c_void_p), None) == fp8.FP8_ERR_INVALID_ARG
+    assert fp8.raw_status("fp8_rings_fold", S, 3, None, None) == fp8.FP8_ERR_INVALID_ARG
+    bad = (ctypes.c_int32 * 3)(0, 7, 0)
+    assert fp8.raw_status("fp8_rings_fold", S, 3, ctypes.cast(bad, ctypes.c_void_p), None) == fp8.FP8_ERR_INVALID_ARG
+    assert fp8.raw_status("fp8_rings_fold", S + 2, 3, ctypes.cast(arr, ctypes.c_void_p), None) == fp8.FP8_ERR_ALIGNMENT
+    jobs = (fp8.fp8_quantize_job * 1)(fp8.fp8_quantize_job(A, 64, 0, 0, S, A + 4096, None, S + 64))
+    assert fp8.raw_status("fp8_quantize_many_ex", ctypes.cast(jobs, ctypes.c_void_p), 1, 1, None) == \
+        fp8.FP8_ERR_INVALID_ARG  # the seed is not offered for grouped calls

@@ -404,3 +404,101 @@ def test_dual_quantize_empty_and_row_layout(g):
     out, _, _, _ = _q2d(g, x, 0, 96, 40, E4M3, None, 0, fp8.FP8_QL_ROW)
     want, _, _ = oracle.quantize_current(x.float().cpu().numpy().reshape(-1), E4M3)
     assert np.array_equal(g.codes(out), want)
+
+
+# ------------------------------------------- data-parallel amax exchange ---
+
+def _bits(a):
+    return int(np.array([a], np.float32).view(np.int32)[0])
+
+
+def test_deferred_fold_with_a_group_amax(g):
+    """Deferred calls leave each ring's amax in its accumulator; with the
+    group's amax written there (as the all-reduce would) one fp8_rings_fold
+    folds all rings exactly as the oracle folds that amax. Without a remote
+    contribution, deferred + fold equals a plain delayed call bit for bit."""
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    fmts = [E4M3, E4M3, E5M2]
+    rings = torch.zeros(3, 20, dtype=torch.int32, device="cuda")
+    for i in range(3):
+        fp8.fp8_ring_init(rings[i], 1.0)
+    twin = g.new_ring()  # plain delayed calls on ring 0's inputs
+    refs = [oracle.DelayedRing() for _ in fmts]
+    for step in range(4):
+        xs = [(W.bf16_normal((50001 + 8 * i,), 0.02 * (i + 1), 9800 + 10 * step + i).float() * (step + 1))
+              .to(torch.bfloat16) for i in range(3)]
+        locals_ = []
+        for i, x in enumerate(xs):
+            q, amax, scale = g.quantize_ex(x.cuda(), 0, fmts[i], rings[i], fp8.FP8_QUANTIZE_DEFER_FOLD)
+            xf = x.float().numpy()
+            s_used = np.float32(refs[i].scale)
+            assert np.array_equal(g.codes(q), oracle.quantize_with_scale(xf, s_used, fmts[i])), (step, i)
+            assert g.f32(scale)[0] == s_used and g.f32(amax)[0] == oracle.amax(xf)
+            locals_.append(np.float32(oracle.amax(xf)))
+        # the all-reduce: another rank saw 3x the amax of role 1 (and less for role 2)
+        group = [locals_[0], np.float32(locals_[1] * 3), locals_[2]]
+        assert int(rings[1, 18]) == _bits(locals_[1])
+        rings[1, 18] = _bits(group[1])
+        rings[2, 18] = max(int(rings[2, 18]), _bits(locals_[2] / 2))
+        fp8.fp8_rings_fold(rings, 3, fmts)
+        for i in range(3):
+            refs[i].fold(group[i], fmts[i])
+            hist, rs, idx, acc, ticket = g.ring_state(rings[i])
+            assert np.array_equal(hist, refs[i].hist) and rs == refs[i].scale and idx == refs[i].idx, (step, i)
+            assert acc == 0 and ticket == 0
+        # ring 0 had no remote contribution: it matches the plain delayed twin
+        q_t, _, s_t = g.quantize(xs[0].cuda(), E4M3, twin)
+        assert np.array_equal(g.ring_state(twin)[0], g.ring_state(rings[0])[0])
+        assert g.ring_state(twin)[1] == g.ring_state(rings[0])[1]
+
+
+def test_grouped_deferred_then_fold(g):
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    sizes = [70001, 4096 * 5, 333]
+    fmts = [E4M3, E5M2, E4M3]
+    rings = torch.zeros(3, 20, dtype=torch.int32, device="cuda")
+    for i in range(3):
+        fp8.fp8_ring_init(rings[i], 1.0)
+    refs = [oracle.DelayedRing() for _ in sizes]
+    outs = [torch.empty(n, dtype=torch.uint8, device="cuda") for n in sizes]
+    scs = [torch.empty(1, device="cuda") for _ in sizes]
+    for step in range(3):
+        xs = [W.bf16_normal((n,), 0.1 * (step + 1), 9900 + 10 * step + j) for j, n in enumerate(sizes)]
+        xd = [x.cuda() for x in xs]
+        fp8.fp8_quantize_many([(xd[j], sizes[j], fmts[j], rings[j], outs[j], None, scs[j]) for j in range(3)],
+                              flags=fp8.FP8_QUANTIZE_DEFER_FOLD)
+        fp8.fp8_rings_fold(rings, 3, fmts)
+        for j in range(3):
+            want, a, s = refs[j].step(xs[j].float().numpy(), fmts[j])
+            assert np.array_equal(g.codes(outs[j]), want) and g.f32(scs[j])[0] == s
+            hist, rs, idx, acc, ticket = g.ring_state(rings[j])
+            assert np.array_equal(hist, refs[j].hist) and rs == refs[j].scale and acc == 0 and ticket == 0
+
+
+def test_exchange_helper_on_one_rank(g):
+    """The torch.distributed helper end to end on a one-rank NCCL group (the
+    all-reduce is then the identity): deferred calls, exchange, fold."""
+    import socket
+    import torch.distributed as dist
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    from fp8_delayed_scaling_quantize_b200.dist import allreduce_amax_and_fold
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1)
+    try:
+        rings = torch.zeros(2, 20, dtype=torch.int32, device="cuda")
+        for i in range(2):
+            fp8.fp8_ring_init(rings[i], 1.0)
+        refs = [oracle.DelayedRing(), oracle.DelayedRing()]
+        x = W.bf16_normal((12345,), 0.3, 9950)
+        for i, fmt in enumerate((E4M3, E5M2)):
+            g.quantize_ex(x.cuda(), 0, fmt, rings[i], fp8.FP8_QUANTIZE_DEFER_FOLD)
+            refs[i].fold(oracle.amax(x.float().numpy()), fmt)
+        allreduce_amax_and_fold(rings, [E4M3, E5M2])
+        torch.cuda.synchronize()
+        for i in range(2):
+            hist, rs, idx, acc, _ = g.ring_state(rings[i])
+            assert np.array_equal(hist, refs[i].hist) and rs == refs[i].scale and acc == 0
+    finally:
+        dist.destroy_process_group()
