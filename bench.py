@@ -184,11 +184,16 @@ class Stack:
             self.sets.append([{k: v.to(dev) for k, v in t.items()} for t in ts])
         T = W.TOKENS
         self.lin = []
+        # all 12 rings in one [12, 20] tensor, so the data-parallel exchange
+        # all-reduces their amax words in one message and folds them in one launch
+        self.rings = torch.empty(3 * len(W.LINEARS), 20, dtype=torch.int32, device=dev)
+        self.ring_fmts = [E4M3, E4M3, E5M2] * len(W.LINEARS)
+        self.dp_amax = False
         for li, (name, d_in, d_out) in enumerate(W.LINEARS):
             L = {"name": name, "d_in": d_in, "d_out": d_out}
             L["q"] = {r: torch.empty(n, dtype=torch.uint8, device=dev)
                       for r, n in (("x", T * d_in), ("w", d_out * d_in), ("g", T * d_out))}
-            L["ring"] = {r: torch.empty(20, dtype=torch.int32, device=dev) for r in ("x", "w", "g")}
+            L["ring"] = {r: self.rings[3 * li + k] for k, r in enumerate(("x", "w", "g"))}
             for r in L["ring"].values():
                 fp8.fp8_ring_init(r, 1.0)
             L["scale"] = {r: torch.empty(1, device=dev) for r in ("x", "w", "g")}
@@ -210,6 +215,24 @@ class Stack:
             need = max(self.fp8.fp8_mm_workspace_size(*c[7:11], c[6], split_k) for li in range(len(self.lin))
                        for c in self.gemm_calls(li))
             self.ws = [torch.zeros(max(need, 4096), dtype=torch.uint8, device=self.dev) for _ in range(2)]
+
+    def quantize(self, call, stream):
+        if self.dp_amax:
+            x, n, fmt, ring, out8, amax, scale = call
+            self.fp8.fp8_quantize_ex(x, 0, n, fmt, ring, self.fp8.FP8_QUANTIZE_DEFER_FOLD, out8, amax, scale,
+                                     stream=stream)
+        else:
+            self.fp8.fp8_quantize(*call, stream=stream)
+
+    def exchange(self, stream):
+        """The data-parallel amax exchange at the end of a step: all-reduce the
+        12 rings' amax words over the ranks (none with one rank), one fold."""
+        import torch.distributed as dist
+        from fp8_delayed_scaling_quantize_b200.dist import allreduce_amax
+        with torch.cuda.stream(stream):
+            if dist.is_initialized() and dist.get_world_size() > 1:
+                allreduce_amax(self.rings)
+            self.fp8.fp8_rings_fold(self.rings, self.rings.shape[0], self.ring_fmts, stream=stream)
 
     def mm(self, call, stream, ws_index=0):
         c = call
@@ -260,26 +283,27 @@ class Stack:
         fp8 = self.fp8
         n = len(self.lin)
         if grouped:
-            fp8.fp8_quantize_many(self.grouped_call(s), stream=stream)
+            fp8.fp8_quantize_many(self.grouped_call(s), stream=stream,
+                                  flags=fp8.FP8_QUANTIZE_DEFER_FOLD if self.dp_amax else 0)
         for li in range(n):
             qx, qw, _ = self.quant_calls(s, li)
             fwd, _, _ = self.gemm_calls(li)
             if grouped:
                 if li > 0:
-                    fp8.fp8_quantize(*qx, stream=stream)
+                    self.quantize(qx, stream)
             elif side is not None:
                 side.wait_stream(stream)
-                fp8.fp8_quantize(*qw, stream=side)
-                fp8.fp8_quantize(*qx, stream=stream)
+                self.quantize(qw, side)
+                self.quantize(qx, stream)
                 stream.wait_stream(side)
             else:
-                fp8.fp8_quantize(*qx, stream=stream)
-                fp8.fp8_quantize(*qw, stream=stream)
+                self.quantize(qx, stream)
+                self.quantize(qw, stream)
             self.mm(fwd, stream)
         for li in reversed(range(n)):
             _, _, qg = self.quant_calls(s, li)
             _, dx, dw = self.gemm_calls(li)
-            fp8.fp8_quantize(*qg, stream=stream)
+            self.quantize(qg, stream)
             if side is not None:
                 side.wait_stream(stream)
                 self.mm(dw, side, 1)
@@ -288,10 +312,12 @@ class Stack:
             else:
                 self.mm(dx, stream)
                 self.mm(dw, stream)
+        if self.dp_amax:
+            self.exchange(stream)
 
     def launches_per_step(self, grouped=True):
         n = len(self.lin)
-        return 3 * n + (1 + (n - 1) + n if grouped else 3 * n)
+        return 3 * n + (1 + (n - 1) + n if grouped else 3 * n) + (1 if self.dp_amax else 0)
 
 
 def hold_stream(stream, us=2000):
@@ -317,6 +343,7 @@ def run_ours(args, world, rank, local):
     side = None if args.one_stream else torch.cuda.Stream()
     stack = Stack(fp8)
     stack.use_split(args.split_k)
+    stack.dp_amax = args.dp_amax
     grouped = not args.no_grouped
     torch.cuda.synchronize()
 
@@ -350,10 +377,12 @@ def run_ours(args, world, rank, local):
                 if graphs:
                     graphs[i % N_SETS].replay()
                 else:
-                    stack.step(i % N_SETS, stream, side)
+                    stack.step(i % N_SETS, stream, side, grouped)
             e1.record(stream)
         e1.synchronize()
     torch.cuda.synchronize()
+    used_graphs = bool(graphs)
+    graphs.clear()  # released before anything else: they may hold NCCL calls (--dp-amax)
     barrier(world)
     t_ms = max_over_ranks(e0.elapsed_time(e1), world)
     ms_step = t_ms / args.steps
@@ -440,14 +469,15 @@ def run_ours(args, world, rank, local):
                    "gemm_gflop_per_step": round(stack.flops / 1e9, 2),
                    "quant_elems_per_step": stack.q_elems,
                    "l2": f"{N_SETS} rotating input sets ({N_SETS * 2 * stack.q_elems / 1e6:.0f} MB bf16) > 126 MB L2",
-                   "launch": ("CUDA graph per step" if graphs else "eager") +
+                   "launch": ("CUDA graph per step" if used_graphs else "eager") +
                              (", 1 stream" if side is None else
                               ", 2 streams (dX||dW" + (")" if grouped else ", x||W quantize)")) +
                              (", all W + first x quantized in one grouped launch" if grouped else "") +
-                             (f", GEMMs split {stack.split_k} ways along K" if stack.split_k > 1 else ""),
+                             (f", GEMMs split {stack.split_k} ways along K" if stack.split_k > 1 else "") +
+                             (", data-parallel amax all-reduce + one ring fold per step" if stack.dp_amax else ""),
                    "launches_per_step": stack.launches_per_step(grouped),
                    "order": "forward over linears, then backward in reverse",
-                   "parallelism": f"replicas x{world}"},
+                   "parallelism": f"replicas x{world}" + (" with the amax all-reduce" if stack.dp_amax else "")},
         "quantize_gbs": round(quant_gbs, 1),
         "roofline": {"bound": "tensor", "achieved": round(gemm_tf, 1), "peak": round(fp8_burst, 1),
                      "unit": "TFLOP/s", "frac": round(gemm_tf / fp8_burst, 4),
@@ -808,6 +838,8 @@ def main():
     ap.add_argument("--one-stream", action="store_true", help="issue the whole step on one stream")
     ap.add_argument("--no-grouped", action="store_true", help="quantize every tensor with its own launch")
     ap.add_argument("--split-k", type=int, default=0, help="force this many K splits in the GEMMs (0: library choice)")
+    ap.add_argument("--dp-amax", action="store_true",
+                    help="deferred ring folds + the ranks' amax all-reduce (MAX) and one fold per step")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-compare", action="store_true", help="skip the bf16 / autograd comparison")
