@@ -59,8 +59,12 @@ from .gemm import (  # noqa: F401
     NN,
     TN,
     mm,
+    mm_exact,
+    mm_out8,
     mm_sampled,
     tolerance,
+    fp8_ulp,
+    out8_tolerance,
 )
 from .linear import (  # noqa: F401
     bias_grad,

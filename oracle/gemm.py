@@ -17,7 +17,10 @@ What the AstrAI commit logs fix:
   one matrix to every batch (``astrai/extension/fp8.py @f4c44ebf``, bullet
   on 3-D mm_fp8 operands).
 * the output is always bf16 (``astrai/extension/fp8.py @f4c44ebf``, bullet
-  dropping the fp8 output parameter).
+  dropping the fp8 output parameter); the FP8-in / FP8-out op that an earlier
+  page adds (``tests/extension/test_fp8_mma.py @cebdd45d``, bullet on
+  fp8_mm_prequant_fp8) is ``mm_out8``: the same y, rounded once to fp32, then
+  quantized with the output scale as a quantize call would.
 
 Definition written out (all matrices row-major, codes decoded exactly):
 
@@ -80,23 +83,66 @@ def _bias64(bias, bias_scale, bias_fmt, N):
     return _decoded(bias.astype(np.uint8), bias_fmt) / np.float64(np.float32(bias_scale))
 
 
-def mm(a8, fa, b8, fb, sa, sb, layout, M, N, K, batch=1, stride_a=None,
-       stride_b=None, bias=None, bias_scale=None, bias_fmt=0):
-    """Full GEMM. Returns (y [batch,M,N] bf16 values as fp32,
-    abs_sum [batch,M,N] = sum_k |A B| / (sa sb) as fp64)."""
+def mm_exact(a8, fa, b8, fb, sa, sb, layout, M, N, K, batch=1, stride_a=None,
+             stride_b=None, bias=None, bias_scale=None, bias_fmt=0):
+    """The GEMM before any output rounding. Returns (y [batch,M,N] =
+    d / (sa sb) + bias in fp64, abs_sum [batch,M,N] = sum_k |A B| / (sa sb))."""
     stride_a = M * K if stride_a is None else stride_a
     stride_b = N * K if stride_b is None else stride_b
     inv = 1.0 / (np.float64(np.float32(sa)) * np.float64(np.float32(sb)))
     bias64 = _bias64(bias, bias_scale, bias_fmt, N)
-    y = np.empty((batch, M, N), dtype=np.float32)
+    y = np.empty((batch, M, N), dtype=np.float64)
     s = np.empty((batch, M, N), dtype=np.float64)
     for b in range(batch):
         A = _op_a(a8, fa, layout, M, K, b, stride_a)
         B = _op_b(b8, fb, layout, N, K, b, stride_b)
-        d = A @ B
-        y[b] = bf16_round_from_f64(d * inv + bias64[None, :])
+        y[b] = (A @ B) * inv + bias64[None, :]
         s[b] = (np.abs(A) @ np.abs(B)) * inv
     return y, s
+
+
+def mm(a8, fa, b8, fb, sa, sb, layout, M, N, K, batch=1, stride_a=None,
+       stride_b=None, bias=None, bias_scale=None, bias_fmt=0):
+    """Full GEMM. Returns (y [batch,M,N] bf16 values as fp32,
+    abs_sum [batch,M,N] = sum_k |A B| / (sa sb) as fp64)."""
+    y64, s = mm_exact(a8, fa, b8, fb, sa, sb, layout, M, N, K, batch, stride_a, stride_b, bias, bias_scale,
+                      bias_fmt)
+    return bf16_round_from_f64(y64).astype(np.float32), s
+
+
+def mm_out8(a8, fa, b8, fb, sa, sb, layout, M, N, K, out_fmt, out_scale, batch=1, stride_a=None,
+            stride_b=None, bias=None, bias_scale=None, bias_fmt=0):
+    """FP8-output GEMM: y as in ``mm`` rounded once to fp32, then
+    q = sat_rne(fp32(y * out_scale)) (``quantize_with_scale``). Returns
+    (codes [batch,M,N] uint8, y64 [batch,M,N], abs_sum [batch,M,N],
+    amax = max |fp32(y)|)."""
+    from .quantize import amax, quantize_with_scale
+    y64, s = mm_exact(a8, fa, b8, fb, sa, sb, layout, M, N, K, batch, stride_a, stride_b, bias, bias_scale,
+                      bias_fmt)
+    y32 = y64.astype(np.float32)
+    q = quantize_with_scale(y32.reshape(-1), np.float32(out_scale), out_fmt).reshape(y32.shape)
+    return q, y64, s, amax(y32.reshape(-1))
+
+
+def fp8_ulp(v, fmt):
+    """Spacing of the FP8 values of ``fmt`` at magnitude |v| (the subnormal
+    spacing below the smallest normal): 2^(max(e, emin) - mantissa bits)."""
+    mbits, emin = (3, -6) if fmt == 0 else (2, -14)
+    a = np.abs(np.asarray(v, dtype=np.float64))
+    _, ex = np.frexp(np.where(a > 0, a, 1.0))
+    e = np.where(a > 0, np.maximum(ex - 1, emin), emin)
+    return np.ldexp(1.0, e - mbits)
+
+
+def out8_tolerance(y64, abs_sum, out_scale, fmt):
+    """Allowed |dec(q_gpu) - clamp(y64 * s)| for an FP8-output GEMM: one FP8
+    spacing at the clamped target plus the GEMM's own error bound (2^-16 of
+    the scaled absolute sum, and one fp32 rounding of y), scaled by s."""
+    fmax = 448.0 if fmt == 0 else 57344.0
+    s = np.float64(np.float32(out_scale))
+    t = np.clip(np.asarray(y64, np.float64) * s, -fmax, fmax)
+    err = (2.0 ** -16 * np.asarray(abs_sum, np.float64) + 2.0 ** -23 * np.abs(y64)) * s
+    return t, fp8_ulp(t, fmt) + err
 
 
 def mm_sampled(a8, fa, b8, fb, sa, sb, layout, M, N, K, idx, batch=1,

@@ -16,6 +16,7 @@ import torch
 import oracle
 from oracle import E4M3, E5M2, NN, NT, TN
 from workloads import fp8_codes
+import workloads as W
 
 TORCH_FP8 = {E4M3: torch.float8_e4m3fn, E5M2: torch.float8_e5m2}
 
@@ -152,3 +153,38 @@ def test_tolerance_ulp_points():
     t = oracle.tolerance(np.array([1.0, 1.5, -3.0, 2.0 ** -130, 0.0, 256.0]), np.zeros(6))
     assert list(t) == [2.0 ** -7, 2.0 ** -7, 2.0 ** -6, 2.0 ** -133, 2.0 ** -133, 2.0]
     assert oracle.tolerance(np.array([0.0]), np.array([2.0 ** 16]))[0] == 1.0 + 2.0 ** -133
+
+
+def test_mm_out8_identity_and_composition():
+    """An identity A passes B's values through exactly (scale 1, no bias), so
+    the FP8 output reproduces B's codes for every finite non-negative-zero
+    code of the same format; with a scale and a bias the codes are the quantize
+    of fp32(y); the amax is max |fp32(y)|."""
+    M = N = K = 32
+    for fmt in (E4M3, E5M2):
+        one = int(np.nonzero(oracle.decode_table(fmt) == 1.0)[0][0])
+        a = np.zeros((M, K), np.uint8)
+        a[np.arange(M), np.arange(K)] = one
+        b = W.fp8_codes((K * N,), fmt, 41 + fmt).numpy()
+        b[b == 0x80] = 0  # -0 sums to +0
+        q, y64, s, amax = oracle.mm_out8(a.reshape(-1), fmt, b, fmt, 1.0, 1.0, NN, M, N, K, fmt, 1.0)
+        assert np.array_equal(q[0].reshape(-1), b)
+        assert amax == np.max(np.abs(oracle.decode_table(fmt)[b]))
+    # composition with a scale and a bf16 bias
+    a8 = W.fp8_codes((64 * 96,), E4M3, 51).numpy()
+    b8 = W.fp8_codes((80 * 96,), E4M3, 52).numpy()
+    bias = W.bf16_normal((80,), 0.5, 53).view(torch.int16).numpy().view(np.uint16)
+    q, y64, s, amax = oracle.mm_out8(a8, E4M3, b8, E4M3, 0.75, 2.0, NT, 64, 80, 96, E5M2, 3.5, bias=bias)
+    y32 = y64.astype(np.float32)
+    assert np.array_equal(q.reshape(-1), oracle.quantize_with_scale(y32.reshape(-1), np.float32(3.5), E5M2))
+    assert amax == np.max(np.abs(y32))
+    yb, _ = oracle.mm(a8, E4M3, b8, E4M3, 0.75, 2.0, NT, 64, 80, 96, bias=bias)
+    assert np.array_equal(yb, oracle.bf16_round_from_f64(y64).astype(np.float32))
+
+
+def test_fp8_ulp_points():
+    assert oracle.fp8_ulp(448.0, E4M3) == 32.0          # 1.75 * 2^8: spacing 2^(8-3)
+    assert oracle.fp8_ulp(1.0, E4M3) == 0.125
+    assert oracle.fp8_ulp(2.0 ** -10, E4M3) == 2.0 ** -9  # subnormal spacing
+    assert oracle.fp8_ulp(0.0, E5M2) == 2.0 ** -16
+    assert oracle.fp8_ulp(57344.0, E5M2) == 2.0 ** 13   # 1.75 * 2^15
