@@ -82,6 +82,7 @@ def _load():
         "fp8_mm_ws": (I, [P, I, P, I, P, P, I, I64, I64, I64, I64, I64, I64, I64, P, P, I, P, P, ctypes.c_size_t,
                           ctypes.c_int32, P]),
         "fp8_mm_workspace_size": (ctypes.c_size_t, [I64, I64, I64, I64, I, ctypes.c_int32]),
+        "fp8_mm_out8": (I, [P, I, P, I, P, P, I, I64, I64, I64, I64, I64, I64, I64, P, P, I, I, P, P, P, P, P]),
         "fp8_mm_splitk_static": (I, [P, I, P, I, P, P, I, I64, I64, I64, I64, I64, I64, I64, P, P, I, P,
                                      ctypes.c_int32, P]),
     }
@@ -198,6 +199,14 @@ def fp8_mm_ws(a8, fa, b8, fb, sa, sb, layout, M, N, K, batch, stride_a, stride_b
                                 int(M), int(N), int(K), int(batch), int(stride_a), int(stride_b),
                                 int(stride_c), _ptr(bias), _ptr(bias_scale), int(bias_fmt), _ptr(out),
                                 _ptr(workspace), int(workspace_bytes), int(split_k), _stream(stream)), "fp8_mm_ws")
+
+
+def fp8_mm_out8(a8, fa, b8, fb, sa, sb, layout, M, N, K, batch, stride_a, stride_b, stride_c, bias,
+                bias_scale, bias_fmt, out_fmt, out_ring, out8, out_amax, out_scale, stream=None):
+    return _check(lib.fp8_mm_out8(_ptr(a8), int(fa), _ptr(b8), int(fb), _ptr(sa), _ptr(sb), int(layout),
+                                  int(M), int(N), int(K), int(batch), int(stride_a), int(stride_b), int(stride_c),
+                                  _ptr(bias), _ptr(bias_scale), int(bias_fmt), int(out_fmt), _ptr(out_ring),
+                                  _ptr(out8), _ptr(out_amax), _ptr(out_scale), _stream(stream)), "fp8_mm_out8")
 
 
 def fp8_mm_workspace_size(M, N, K, batch, layout, split_k):

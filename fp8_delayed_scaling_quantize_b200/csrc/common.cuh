@@ -63,4 +63,37 @@ __device__ __forceinline__ float scale_from_amax(float fmax, float m) {
     return isinf(s) ? 3.402823466e38f : s;
 }
 
+// The delayed-scaling fold of amax `a` into a ring [fp8.py@4dc5e923, bullet
+// on the last-block epilogue]: hist[idx] = a, idx advances, and the window's
+// maximum (the 15 kept entries and a) publishes fmt_max / max when it is
+// finite and > 0 (otherwise the scale is kept). hist and idx must be the
+// values read by the caller (h[], idx), which lets it issue those reads
+// early.
+__device__ __forceinline__ void ring_fold(volatile fp8_ring* r, const float (&h)[FP8_RING_HISTORY], uint32_t idx,
+                                          float a, float fmax) {
+    float wmax = a;
+#pragma unroll
+    for (int i = 0; i < FP8_RING_HISTORY; ++i)
+        if (uint32_t(i) != idx) wmax = fmaxf(wmax, h[i]);
+    r->hist[idx] = a;
+    if (wmax > 0.0f && isfinite(wmax)) r->scale = scale_from_amax(fmax, wmax);
+    r->idx = (idx + 1) & (FP8_RING_HISTORY - 1);
+}
+
+// Atomic add with acquire-release semantics at GPU scope (the last-block
+// election of a ring finalize: a block's earlier amax publication is visible
+// before its ticket moves, and the block drawing the last ticket sees all).
+__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
+// Reads a ring's history and index (for ring_fold).
+__device__ __forceinline__ uint32_t ring_read(volatile fp8_ring* r, float (&h)[FP8_RING_HISTORY]) {
+#pragma unroll
+    for (int i = 0; i < FP8_RING_HISTORY; ++i) h[i] = r->hist[i];
+    return r->idx & (FP8_RING_HISTORY - 1);
+}
+
 }  // namespace fp8lite

@@ -80,6 +80,11 @@ struct GemmParams {
     int split, kb_per, total_units;
     float* ws;         // fp32 partial slots: [tile][rank][split] x (128 x BN)
     uint32_t* ws_cnt;  // per (tile, rank): {units arrived, partials written}
+    // FP8 output (fp8_mm_out8): format, delayed-scaling ring, the scale used, the amax
+    int out_fmt;
+    fp8_ring* out_ring;
+    float* out_scale;
+    float* out_amax;
 };
 
 // Wait for phase `parity` of the mbarrier at `bar`, giving up after
@@ -141,6 +146,15 @@ __device__ __forceinline__ float fp8_to_f32(uint8_t c, int fmt) {
         asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h) : "h"(in));
     }
     return __half2float(__ushort_as_half(uint16_t(h & 0xFFFFu)));
+}
+
+// Two fp32 values to a pair of FP8 codes (nearest-even, saturating), the
+// first in the low byte.
+__device__ __forceinline__ uint32_t cvt_fp8x2(int fmt, float lo, float hi) {
+    uint16_t r;
+    if (fmt == FP8_E4M3) asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    else                 asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -230,7 +244,7 @@ __device__ __forceinline__ bool epilogue_bar_or(bool v) {
 // Epilogue: 4 warps, one per TMEM lane quarter. Every 32 columns of the tile
 // become a 128 x 32 bf16 tile in shared memory that one thread writes with a
 // single TMA store (8 stores for a 128 x 256 tile).
-template <int BN, bool A_MN, bool B_MN, int STAGES, bool HAS_BIAS, int CTAS, bool SPLIT, bool SWAP>
+template <int BN, bool A_MN, bool B_MN, int STAGES, bool HAS_BIAS, int CTAS, bool SPLIT, bool SWAP, bool OUT8>
 __global__ void __maxnreg__(168)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const __grid_constant__ CUtensorMap tm_c, const GemmParams p) {
@@ -393,6 +407,13 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         int n_st = 0;  // TMA stores issued so far (they alternate between the two staging tiles)
         const float inv = (1.0f / __ldg(p.sa)) * (1.0f / __ldg(p.sb));
         const float bscale = (HAS_BIAS && p.bias_kind == 2) ? __ldg(p.bias_scale) : 1.0f;
+        // FP8 output: the ring's scale before this call (every CTA reads it
+        // before any CTA can fold: the fold waits for all CTAs' tickets)
+        float s_out = 1.0f, m_out = 0.0f;
+        if (OUT8) {
+            s_out = *reinterpret_cast<volatile float*>(&p.out_ring->scale);
+            if (blockIdx.x == 0 && etid == 0) *p.out_scale = s_out;
+        }
         bool failed = false;
         int it = 0;
         for (int u = unit0; u < total_units; u += unit_step, ++it) {
@@ -538,7 +559,32 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                         const float bias = HAS_BIAS ? s_bias[c * CW + i] : 0.0f;
                         y[i] = fmaf(__uint_as_float(r[i]), inv, bias);
                     }
-                    if (tma_store) {
+                    if constexpr (OUT8) {
+                        // q = sat_rne(fp32(y * s_out)); the amax is over the
+                        // unquantized y of this call's own outputs only
+                        if (row < M) {
+                            uint32_t w[8];
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+#pragma unroll
+                                for (int k = 0; k < 4; ++k)
+                                    if (col0 + 4 * j + k < N) m_out = fmaxf(m_out, fabsf(y[4 * j + k]));
+                                w[j] = cvt_fp8x2(p.out_fmt, __fmul_rn(y[4 * j], s_out), __fmul_rn(y[4 * j + 1], s_out)) |
+                                       (cvt_fp8x2(p.out_fmt, __fmul_rn(y[4 * j + 2], s_out),
+                                                  __fmul_rn(y[4 * j + 3], s_out)) << 16);
+                            }
+                            uint8_t* dst = reinterpret_cast<uint8_t*>(p.out) + int64_t(b) * p.stride_c +
+                                           int64_t(row) * N + col0;
+                            if (vec_store && col0 + 32 <= N) {
+                                reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                                reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                            } else {
+#pragma unroll
+                                for (int i = 0; i < 32; ++i)
+                                    if (col0 + i < N) dst[i] = uint8_t(w[i >> 2] >> (8 * (i & 3)));
+                            }
+                        }
+                    } else if (tma_store) {
                         // the 128 x 32 bf16 block goes to the staging tile whose last
                         // store is known to have read it (64-byte swizzle: 16-byte
                         // piece j of row r at (j ^ (r / 2 mod 4)) * 16, so the 8
@@ -597,6 +643,30 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         // writes themselves complete with the grid (a dependent kernel's
         // griddepcontrol.wait and stream order both see them)
         if (tma_store && store_lead) bulk_wait_read<0>();
+        if constexpr (OUT8) {
+            // the CTA's amax of the output: one atomicMax, then a ticket; the
+            // CTA holding the last ticket folds it into the output's ring
+            uint32_t bits = __reduce_max_sync(0xffffffffu, __float_as_uint(m_out));
+            epilogue_bar();  // the bias slots are free now
+            uint32_t* red = reinterpret_cast<uint32_t*>(s_bias);
+            if (lane == 0) red[q] = bits;
+            epilogue_bar();
+            if (etid == 0) {
+                bits = max(max(red[0], red[1]), max(red[2], red[3]));
+                fp8_ring* ring = p.out_ring;
+                if (bits != 0u) atomicMax(&ring->amax_bits, bits);
+                const uint32_t ticket = atom_add_acq_rel(&ring->ticket, 1u);
+                if (ticket == gridDim.x - 1) {
+                    volatile fp8_ring* rr = ring;
+                    float h[FP8_RING_HISTORY];
+                    const uint32_t idx = ring_read(rr, h);
+                    const float a = __uint_as_float(atomicExch(&ring->amax_bits, 0u));
+                    ring_fold(rr, h, idx, a, fmt_max(p.out_fmt));
+                    if (p.out_amax) *p.out_amax = a;
+                    rr->ticket = 0u;
+                }
+            }
+        }
     }
 
     tc_fence_before();
@@ -685,11 +755,11 @@ struct HostArgs {
     int64_t batch, stride_b;
 };
 
-template <int BN, bool A_MN, bool B_MN, int STAGES, bool HAS_BIAS, int CTAS, bool SPLIT, bool SWAP>
+template <int BN, bool A_MN, bool B_MN, int STAGES, bool HAS_BIAS, int CTAS, bool SPLIT, bool SWAP, bool OUT8>
 fp8_status launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, GemmParams p,
                       const HostArgs& h, cudaStream_t st) {
     using L = Smem<BN, STAGES, CTAS>;
-    auto kern = fp8_gemm_kernel<BN, A_MN, B_MN, STAGES, HAS_BIAS, CTAS, SPLIT, SWAP>;
+    auto kern = fp8_gemm_kernel<BN, A_MN, B_MN, STAGES, HAS_BIAS, CTAS, SPLIT, SWAP, OUT8>;
     static bool attr_set[64] = {false};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8_ERR_CUDA;
@@ -712,15 +782,21 @@ fp8_status launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
     return launch_pdl(kern, units * CTAS, kThreads, L::kAlloc, st, CTAS, ta, tb, tc, p);
 }
 
-template <int BN, bool A_MN, bool B_MN, int STAGES, int CTAS, bool SWAP = false>
+template <int BN, bool A_MN, bool B_MN, int STAGES, int CTAS, bool SWAP = false, bool OUT8 = false>
 fp8_status launch(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, const HostArgs& h, cudaStream_t st) {
     CUtensorMap tc = {};
     if (p.tma_store && !make_out_map(&tc, p.out, p.N, p.M, h.batch, uint64_t(p.stride_c) * 2)) return FP8_ERR_CUDA;
-    if (p.split > 1)
-        return p.bias_kind ? launch_one<BN, A_MN, B_MN, STAGES, true, CTAS, true, SWAP>(ta, tb, tc, p, h, st)
-                           : launch_one<BN, A_MN, B_MN, STAGES, false, CTAS, true, SWAP>(ta, tb, tc, p, h, st);
-    return p.bias_kind ? launch_one<BN, A_MN, B_MN, STAGES, true, CTAS, false, SWAP>(ta, tb, tc, p, h, st)
-                       : launch_one<BN, A_MN, B_MN, STAGES, false, CTAS, false, SWAP>(ta, tb, tc, p, h, st);
+    if constexpr (OUT8) {  // no split, no swap
+        return p.bias_kind ? launch_one<BN, A_MN, B_MN, STAGES, true, CTAS, false, false, true>(ta, tb, tc, p, h, st)
+                           : launch_one<BN, A_MN, B_MN, STAGES, false, CTAS, false, false, true>(ta, tb, tc, p, h, st);
+    } else {
+        if (p.split > 1)
+            return p.bias_kind
+                       ? launch_one<BN, A_MN, B_MN, STAGES, true, CTAS, true, SWAP, false>(ta, tb, tc, p, h, st)
+                       : launch_one<BN, A_MN, B_MN, STAGES, false, CTAS, true, SWAP, false>(ta, tb, tc, p, h, st);
+        return p.bias_kind ? launch_one<BN, A_MN, B_MN, STAGES, true, CTAS, false, SWAP, false>(ta, tb, tc, p, h, st)
+                           : launch_one<BN, A_MN, B_MN, STAGES, false, CTAS, false, SWAP, false>(ta, tb, tc, p, h, st);
+    }
 }
 
 // Tile choice for 148 SMs by a small cost model: a persistent grid walks
@@ -786,7 +862,7 @@ inline TileChoice choose_tile(int64_t M, int64_t N, int64_t K, int64_t batch, bo
     return best;
 }
 
-template <bool A_MN, bool B_MN>
+template <bool A_MN, bool B_MN, bool OUT8 = false>
 fp8_status dispatch(const CUtensorMap& ta, GemmParams p, const HostArgs& h, void* ws, size_t ws_bytes,
                     int split_req, cudaStream_t st) {
     const TileChoice tc = choose_tile(p.M, p.N, p.K, h.batch, B_MN, sm_count(), split_req);
@@ -806,10 +882,10 @@ fp8_status dispatch(const CUtensorMap& ta, GemmParams p, const HostArgs& h, void
     const bool ok = B_MN ? make_map(&tb, h.b8, p.N, p.K, h.batch, sb_bytes, 128, BK)
                          : make_map(&tb, h.b8, p.K, p.N, h.batch, sb_bytes, BK, b_box_n);
     if (!ok) return FP8_ERR_CUDA;
-    if (pair) return launch<256, A_MN, B_MN, 6, 2>(ta, tb, p, h, st);
-    if (bn == 256) return launch<256, A_MN, B_MN, 4, 1>(ta, tb, p, h, st);
-    if (bn == 128) return launch<128, A_MN, B_MN, 6, 1>(ta, tb, p, h, st);
-    if constexpr (!B_MN) return launch<64, A_MN, B_MN, 8, 1>(ta, tb, p, h, st);
+    if (pair) return launch<256, A_MN, B_MN, 6, 2, false, OUT8>(ta, tb, p, h, st);
+    if (bn == 256) return launch<256, A_MN, B_MN, 4, 1, false, OUT8>(ta, tb, p, h, st);
+    if (bn == 128) return launch<128, A_MN, B_MN, 6, 1, false, OUT8>(ta, tb, p, h, st);
+    if constexpr (!B_MN) return launch<64, A_MN, B_MN, 8, 1, false, OUT8>(ta, tb, p, h, st);
     return FP8_ERR_UNSUPPORTED;
 }
 
@@ -893,11 +969,23 @@ fp8_status dispatch_swap(const uint8_t* a8, int fa, const uint8_t* b8, int fb, i
 
 using namespace fp8lite;
 
-extern "C" fp8_status fp8_mm_ws(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8, fp8_fmt fb, const float* sa,
-                                const float* sb, fp8_layout layout, int64_t M, int64_t N, int64_t K, int64_t batch,
-                                int64_t stride_a, int64_t stride_b, int64_t stride_c, const void* bias,
-                                const float* bias_scale, fp8_fmt bias_fmt, void* out, void* workspace,
-                                size_t workspace_bytes, int32_t split_k, void* stream) {
+namespace fp8lite {
+namespace {
+
+// The FP8 output of fp8_mm_out8 (none for the bf16 entry points).
+struct Out8 {
+    bool on;
+    fp8_fmt fmt;
+    fp8_ring* ring;
+    float* amax;
+    float* scale;
+};
+
+fp8_status mm_impl(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8, fp8_fmt fb, const float* sa, const float* sb,
+                   fp8_layout layout, int64_t M, int64_t N, int64_t K, int64_t batch, int64_t stride_a,
+                   int64_t stride_b, int64_t stride_c, const void* bias, const float* bias_scale, fp8_fmt bias_fmt,
+                   void* out, void* workspace, size_t workspace_bytes, int32_t split_k, const Out8& o8,
+                   void* stream) {
     if (split_k < 0 || split_k > kMaxSplit) return FP8_ERR_INVALID_ARG;
     if (workspace && !aligned(workspace, 16)) return FP8_ERR_ALIGNMENT;
     if (!valid_fmt(fa) || !valid_fmt(fb)) return FP8_ERR_INVALID_ARG;
@@ -907,6 +995,7 @@ extern "C" fp8_status fp8_mm_ws(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8
     if (stride_a < 0 || stride_b < 0 || stride_c < 0) return FP8_ERR_INVALID_ARG;
     if (bias_scale && !bias) return FP8_ERR_INVALID_ARG;
     if (bias && bias_scale && !valid_fmt(bias_fmt)) return FP8_ERR_INVALID_ARG;
+    if (o8.on && (!valid_fmt(o8.fmt) || !o8.ring || !o8.scale)) return FP8_ERR_INVALID_ARG;
     if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31) ||
         batch >= (int64_t(1) << 31))
         return FP8_ERR_UNSUPPORTED;
@@ -922,8 +1011,9 @@ extern "C" fp8_status fp8_mm_ws(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8
     if (a_pitch % 16 != 0 || b_pitch % 16 != 0) return FP8_ERR_ALIGNMENT;
     if (!aligned(a8, 16) || !aligned(b8, 16)) return FP8_ERR_ALIGNMENT;
     if (stride_a % 16 != 0 || stride_b % 16 != 0) return FP8_ERR_ALIGNMENT;
-    if (!aligned(out, 4) || !aligned(sa, 4) || !aligned(sb, 4)) return FP8_ERR_ALIGNMENT;
+    if (!aligned(out, o8.on ? 1 : 4) || !aligned(sa, 4) || !aligned(sb, 4)) return FP8_ERR_ALIGNMENT;
     if (bias && !bias_scale && !aligned(bias, 2)) return FP8_ERR_ALIGNMENT;
+    if (o8.on && (!aligned(o8.ring, 4) || !aligned(o8.scale, 4) || !aligned(o8.amax, 4))) return FP8_ERR_ALIGNMENT;
     if (batch == 1) { stride_a = 0; stride_b = 0; }
 
     GemmParams p = {};
@@ -942,10 +1032,19 @@ extern "C" fp8_status fp8_mm_ws(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8
     p.out = static_cast<uint16_t*>(out);
     p.stride_c = stride_c;
     p.split = 1;
-    p.vec_store = (N % 8 == 0) && (stride_c % 8 == 0) && aligned(out, 16);
-    p.tma_store = p.vec_store;
+    if (o8.on) {  // byte codes, 16-byte vector stores where rows allow
+        p.out_fmt = int(o8.fmt);
+        p.out_ring = o8.ring;
+        p.out_amax = o8.amax;
+        p.out_scale = o8.scale;
+        p.vec_store = (N % 16 == 0) && (stride_c % 16 == 0) && aligned(out, 16);
+        p.tma_store = 0;
+    } else {
+        p.vec_store = (N % 8 == 0) && (stride_c % 8 == 0) && aligned(out, 16);
+        p.tma_store = p.vec_store;
+    }
     cudaStream_t st = as_stream(stream);
-    if (swap_ab(M, N, layout))
+    if (!o8.on && swap_ab(M, N, layout))
         return layout == FP8_NN ? dispatch_swap<true>(a8, fa, b8, fb, M, N, K, batch, stride_a, stride_b, p, workspace,
                                                       workspace_bytes, split_k, st)
                                 : dispatch_swap<false>(a8, fa, b8, fb, M, N, K, batch, stride_a, stride_b, p,
@@ -956,11 +1055,41 @@ extern "C" fp8_status fp8_mm_ws(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8
                    : make_map(&ta, a8, K, M, batch, uint64_t(stride_a), BK, BM);
     if (!ok) return FP8_ERR_CUDA;
     const HostArgs h = {int(fa), int(fb), b8, batch, stride_b};
+    if (o8.on) {
+        switch (layout) {
+            case FP8_NT: return dispatch<false, false, true>(ta, p, h, nullptr, 0, 1, st);
+            case FP8_NN: return dispatch<false, true, true>(ta, p, h, nullptr, 0, 1, st);
+            default:     return dispatch<true, true, true>(ta, p, h, nullptr, 0, 1, st);
+        }
+    }
     switch (layout) {
         case FP8_NT: return dispatch<false, false>(ta, p, h, workspace, workspace_bytes, split_k, st);
         case FP8_NN: return dispatch<false, true>(ta, p, h, workspace, workspace_bytes, split_k, st);
         default:     return dispatch<true, true>(ta, p, h, workspace, workspace_bytes, split_k, st);
     }
+}
+
+}  // namespace
+}  // namespace fp8lite
+
+extern "C" fp8_status fp8_mm_ws(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8, fp8_fmt fb, const float* sa,
+                                const float* sb, fp8_layout layout, int64_t M, int64_t N, int64_t K, int64_t batch,
+                                int64_t stride_a, int64_t stride_b, int64_t stride_c, const void* bias,
+                                const float* bias_scale, fp8_fmt bias_fmt, void* out, void* workspace,
+                                size_t workspace_bytes, int32_t split_k, void* stream) {
+    const Out8 none = {false, FP8_E4M3, nullptr, nullptr, nullptr};
+    return mm_impl(a8, fa, b8, fb, sa, sb, layout, M, N, K, batch, stride_a, stride_b, stride_c, bias, bias_scale,
+                   bias_fmt, out, workspace, workspace_bytes, split_k, none, stream);
+}
+
+extern "C" fp8_status fp8_mm_out8(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8, fp8_fmt fb, const float* sa,
+                                  const float* sb, fp8_layout layout, int64_t M, int64_t N, int64_t K, int64_t batch,
+                                  int64_t stride_a, int64_t stride_b, int64_t stride_c, const void* bias,
+                                  const float* bias_scale, fp8_fmt bias_fmt, fp8_fmt out_fmt, fp8_ring* out_ring,
+                                  uint8_t* out8, float* out_amax, float* out_scale, void* stream) {
+    const Out8 o8 = {true, out_fmt, out_ring, out_amax, out_scale};
+    return mm_impl(a8, fa, b8, fb, sa, sb, layout, M, N, K, batch, stride_a, stride_b, stride_c, bias, bias_scale,
+                   bias_fmt, out8, nullptr, 0, 1, o8, stream);
 }
 
 extern "C" fp8_status fp8_mm(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8, fp8_fmt fb, const float* sa,

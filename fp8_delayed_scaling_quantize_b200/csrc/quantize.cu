@@ -133,11 +133,6 @@ __device__ __forceinline__ void amax8(const float (&f)[8], float& m) {
     for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
 }
 
-__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
-    uint32_t old;
-    asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-    return old;
-}
 
 // Block-wide max of a non-negative, non-NaN float; result valid in thread 0.
 __device__ __forceinline__ uint32_t block_max_bits(float m) {
@@ -189,19 +184,10 @@ __device__ __forceinline__ void finish_block(float m, fp8_ring* ring, uint32_t* 
     // accesses leave at once and cost one round trip to L2.
     volatile fp8_ring* r = ring;
     float h[FP8_RING_HISTORY];
-#pragma unroll
-    for (int i = 0; i < FP8_RING_HISTORY; ++i) h[i] = r->hist[i];
-    const uint32_t idx = r->idx & (FP8_RING_HISTORY - 1);
+    const uint32_t idx = ring_read(r, h);
     const float a = MODE == kDelayed ? __uint_as_float(atomicExch(&ring->amax_bits, 0u))
                                      : __uint_as_float(*reinterpret_cast<volatile uint32_t*>(amax_acc));
-    // the window's maximum over the 15 kept entries and the new amax
-    float wmax = a;
-#pragma unroll
-    for (int i = 0; i < FP8_RING_HISTORY; ++i)
-        if (uint32_t(i) != idx) wmax = fmaxf(wmax, h[i]);
-    r->hist[idx] = a;
-    if (wmax > 0.0f && isfinite(wmax)) r->scale = scale_from_amax(fmax, wmax);
-    r->idx = (idx + 1) & (FP8_RING_HISTORY - 1);
+    ring_fold(r, h, idx, a, fmax);
     if (MODE == kDelayed) {
         if (amax_out) *amax_out = a;
         r->ticket = 0u;  // ready for the next call (visible at the kernel boundary)
@@ -452,15 +438,9 @@ __global__ void rings_fold_kernel(fp8_ring* rings, int count, const __grid_const
     const int i = threadIdx.x;
     if (i < count) {
         volatile fp8_ring* r = rings + i;
-        const float a = __uint_as_float(r->amax_bits);
-        const uint32_t idx = r->idx & (FP8_RING_HISTORY - 1);
-        float wmax = a;
-#pragma unroll
-        for (int k = 0; k < FP8_RING_HISTORY; ++k)
-            if (uint32_t(k) != idx) wmax = fmaxf(wmax, r->hist[k]);
-        r->hist[idx] = a;
-        if (wmax > 0.0f && isfinite(wmax)) r->scale = scale_from_amax(fmt_max(f.fmt[i]), wmax);
-        r->idx = (idx + 1) & (FP8_RING_HISTORY - 1);
+        float h[FP8_RING_HISTORY];
+        const uint32_t idx = ring_read(r, h);
+        ring_fold(r, h, idx, __uint_as_float(r->amax_bits), fmt_max(f.fmt[i]));
         r->amax_bits = 0u;
     }
     griddep_launch();

@@ -303,6 +303,34 @@ FP8LITE_API fp8_status fp8_mm_ws(const uint8_t* a8, fp8_fmt fa, const uint8_t* b
                   void* out, void* workspace, size_t workspace_bytes, int32_t split_k,
                   void* stream);
 
+/* FP8-in / FP8-out GEMM with delayed output scaling [mma@cebdd45d, bullet on
+ * the fp8_mm_prequant_fp8 custom op for FP8-in/FP8-out GEMM; the later
+ * fp8.py@f4c44ebf page drops that output for bf16 only, so it is an extra
+ * entry point and fp8_mm stays bf16]:
+ *
+ *   y[b,i,j]   = (sum_k op(A_b)[i,k] op(B_b)[k,j]) / (sa*sb) + bias_j   (fp32,
+ *                exactly as fp8_mm computes it before its bf16 rounding)
+ *   out8[b,i,j] = sat_rne_out_fmt( fp32(y[b,i,j] * s) ),  s = out_ring->scale
+ *                as it stood before the call (reported in *out_scale)
+ *
+ * out_ring is a delayed-scaling ring for the output: the amax of |y| over all
+ * outputs (NaN ignored) is folded into it by the last CTA exactly as a
+ * delayed fp8_quantize call folds its input's amax, and reported in
+ * *out_amax (optional). The next layer can use out8 with *out_scale as its
+ * FP8 operand without a separate quantize pass.
+ * All arguments as fp8_mm, except: out8 device uint8[batch*stride_c]
+ * (row-major [M,N] codes of out_fmt per batch; stride_c in elements = bytes);
+ * out_ring required (4-byte aligned); out_scale required. Never splits K and
+ * never swaps operands. Errors as fp8_mm; FP8_ERR_INVALID_ARG also for a bad
+ * out_fmt or a NULL out_ring / out_scale. */
+FP8LITE_API fp8_status fp8_mm_out8(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8, fp8_fmt fb,
+                  const float* sa, const float* sb, fp8_layout layout,
+                  int64_t M, int64_t N, int64_t K, int64_t batch,
+                  int64_t stride_a, int64_t stride_b, int64_t stride_c,
+                  const void* bias, const float* bias_scale, fp8_fmt bias_fmt,
+                  fp8_fmt out_fmt, fp8_ring* out_ring, uint8_t* out8, float* out_amax, float* out_scale,
+                  void* stream);
+
 /* Workspace bytes fp8_mm_ws needs for this problem and split_k on the
  * current device (split_k 0: for the library's own choice): 0 when that call
  * would not split, or for arguments fp8_mm_ws rejects. */

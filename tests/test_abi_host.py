@@ -195,3 +195,14 @@ def test_rings_fold_and_grouped_flags_validation(fmt_ok=(0, 1)):
     jobs = (fp8.fp8_quantize_job * 1)(fp8.fp8_quantize_job(A, 64, 0, 0, S, A + 4096, None, S + 64))
     assert fp8.raw_status("fp8_quantize_many_ex", ctypes.cast(jobs, ctypes.c_void_p), 1, 1, None) == \
         fp8.FP8_ERR_INVALID_ARG  # the seed is not offered for grouped calls
+
+
+def test_mm_out8_validation(fp8):
+    def st(out_fmt=0, ring=S, out8=A + 8192, scale=S + 64, amax=None):
+        return fp8.raw_status("fp8_mm_out8", A, 0, A, 0, S, S, 0, 16, 16, 16, 1, 256, 256, 256, None, None, 0,
+                              out_fmt, ring, out8, amax, scale, None)
+    assert st(out_fmt=3) == fp8.FP8_ERR_INVALID_ARG
+    assert st(ring=None) == fp8.FP8_ERR_INVALID_ARG
+    assert st(scale=None) == fp8.FP8_ERR_INVALID_ARG
+    assert st(out8=None) == fp8.FP8_ERR_INVALID_ARG
+    assert st(ring=S + 2) == fp8.FP8_ERR_ALIGNMENT
