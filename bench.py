@@ -5,12 +5,13 @@ stack at 2048 tokens (B4 x T512): for each of the 4 linears (QKV 1024->3072,
 out 1024->1024, MLP 1024->4096, 4096->1024) delayed-scaling quantize of x
 and W to E4M3 and of the gradient g to E5M2 (ring finalized in-kernel),
 then the forward NT GEMM y = x W^T, the dX NN GEMM g W and the dW TN GEMM
-g^T x, all through the C ABI: 12 GEMM launches and 8 quantize launches (one
-grouped launch for every W and the first x, then each later x and every g;
---no-grouped: 12 single-tensor quantize launches).
+g^T x, all through the C ABI: 8 GEMM launches (a forward per linear, and one
+grouped launch per linear for its dX and dW; --no-group-bwd: 12 single GEMMs)
+and 8 quantize launches (one grouped launch for every W and the first x, then
+each later x and every g; --no-grouped: 12 single-tensor quantize launches).
 
 value  = GEMM FLOPs of the step (154.6 GFLOP) / device step time, TFLOP/s,
-         the step replayed as one CUDA graph (20 kernel nodes), inputs
+         the step replayed as one CUDA graph (16 kernel nodes), inputs
          resident in HBM, rotating through 3 input sets (276 MB > 126 MB L2).
 e2e    = the same metric through the public API with HOST buffers: pinned
          host -> device copies of x, W, g and device -> host copies of y,
@@ -206,6 +207,16 @@ class Stack:
         self.q_elems = W.stack_quant_elems()
         self.split_k = 0
         self.ws = [None, None]
+        self.group_bwd = True
+
+    def use_group_bwd(self):
+        """dX and dW of a linear in one fp8_mm_grouped launch (not with split K)."""
+        return self.group_bwd and self.split_k <= 1
+
+    def bwd_pair(self, li):
+        """dX and dW of linear li as the two problems of one grouped launch."""
+        _, dx, dw = self.gemm_calls(li)
+        return [c[:10] + c[14:18] for c in (dx, dw)]
 
     def use_split(self, split_k):
         """Run every GEMM of the step that can take it with split_k K-splits,
@@ -276,10 +287,12 @@ class Stack:
         grouped: the weights are all known when the step starts, so every W
         and the first x are quantized by one grouped launch; the x of later
         linears and every g still wait for the layer before them.
-        With a `side` stream, the work a linear layer can overlap runs on it:
-        W's quantize beside x's (ungrouped), and dW beside dX (both only need
-        g8); the streams fork and join around each pair, so the dependencies
-        between linears are those of a sequential model."""
+        The backward's dX and dW (both only need g8) run as one grouped GEMM
+        launch; without it (split K, or --no-group-bwd) and with a `side`
+        stream, dW runs on that stream beside dX. A `side` stream also takes
+        W's quantize beside x's (ungrouped). The streams fork and join around
+        each pair, so the dependencies between linears are those of a
+        sequential model."""
         fp8 = self.fp8
         n = len(self.lin)
         if grouped:
@@ -304,7 +317,9 @@ class Stack:
             _, _, qg = self.quant_calls(s, li)
             _, dx, dw = self.gemm_calls(li)
             self.quantize(qg, stream)
-            if side is not None:
+            if self.use_group_bwd():
+                fp8.fp8_mm_grouped(self.bwd_pair(li), stream=stream)
+            elif side is not None:
                 side.wait_stream(stream)
                 self.mm(dw, side, 1)
                 self.mm(dx, stream, 0)
@@ -317,7 +332,8 @@ class Stack:
 
     def launches_per_step(self, grouped=True):
         n = len(self.lin)
-        return 3 * n + (1 + (n - 1) + n if grouped else 3 * n) + (1 if self.dp_amax else 0)
+        gemms = n + (n if self.use_group_bwd() else 2 * n)
+        return gemms + (1 + (n - 1) + n if grouped else 3 * n) + (1 if self.dp_amax else 0)
 
 
 def hold_stream(stream, us=2000):
@@ -344,6 +360,7 @@ def run_ours(args, world, rank, local):
     stack = Stack(fp8)
     stack.use_split(args.split_k)
     stack.dp_amax = args.dp_amax
+    stack.group_bwd = not args.no_group_bwd
     grouped = not args.no_grouped
     torch.cuda.synchronize()
 
@@ -389,16 +406,22 @@ def run_ours(args, world, rank, local):
     value = weak_scaling_value(stack.flops, args.steps, world, t_ms)
 
     # ---- per-kernel breakdown -----------------------------------------
-    # Each of the step's 12 quantizes and 12 GEMMs is repeated back to back between one
-    # event pair (the stream held while the host enqueues), so the average is
-    # the kernel's steady-state cost on the stream, as inside the graph.
+    # Each of the step's 12 quantizes and its GEMM launches (a forward per
+    # linear, and a grouped dX + dW launch per linear, or the two apart) is
+    # repeated back to back between one event pair (the stream held while the
+    # host enqueues), so the average is the kernel's steady-state cost on the
+    # stream, as inside the graph.
     q_ms = g_ms = 0.0
     q_elems = g_flops = g_bytes = 0
     n_g = n_q = 0
     per_shape = {}
     reps = args.breakdown_reps
     for li in range(len(stack.lin)):
-        calls = [("quantize", c) for c in stack.quant_calls(0, li)] + [("gemm", c) for c in stack.gemm_calls(li)]
+        calls = [("quantize", c) for c in stack.quant_calls(0, li)]
+        if stack.use_group_bwd():
+            calls += [("gemm", stack.gemm_calls(li)[0]), ("pair", stack.bwd_pair(li))]
+        else:
+            calls += [("gemm", c) for c in stack.gemm_calls(li)]
         for kind, c in calls:
             hold_stream(stream)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -406,6 +429,8 @@ def run_ours(args, world, rank, local):
             for _ in range(reps):
                 if kind == "quantize":
                     fp8.fp8_quantize(*c, stream=stream)
+                elif kind == "pair":
+                    fp8.fp8_mm_grouped(c, stream=stream)
                 else:
                     stack.mm(c, stream)
             e1.record(stream)
@@ -415,6 +440,13 @@ def run_ours(args, world, rank, local):
                 q_ms += ms
                 q_elems += c[1]
                 n_q += 1
+            elif kind == "pair":
+                g_ms += ms
+                f = sum(2 * M * N * K for (M, N, K) in (q[7:10] for q in c))
+                g_flops += f
+                g_bytes += sum(gemm_algorithmic_bytes(q[6], *q[7:10]) for q in c)
+                n_g += 1
+                per_shape[" + ".join(f"{'NT NN TN'.split()[q[6]]} {q[7]}x{q[8]}x{q[9]}" for q in c)] = (ms, f)
             else:
                 M, N, K = c[7:10]
                 g_ms += ms
@@ -470,7 +502,8 @@ def run_ours(args, world, rank, local):
                    "quant_elems_per_step": stack.q_elems,
                    "l2": f"{N_SETS} rotating input sets ({N_SETS * 2 * stack.q_elems / 1e6:.0f} MB bf16) > 126 MB L2",
                    "launch": ("CUDA graph per step" if used_graphs else "eager") +
-                             (", 1 stream" if side is None else
+                             (", dX + dW of each linear in one grouped GEMM launch" if stack.use_group_bwd() else
+                              ", 1 stream" if side is None else
                               ", 2 streams (dX||dW" + (")" if grouped else ", x||W quantize)")) +
                              (", all W + first x quantized in one grouped launch" if grouped else "") +
                              (f", GEMMs split {stack.split_k} ways along K" if stack.split_k > 1 else "") +
@@ -482,7 +515,8 @@ def run_ours(args, world, rank, local):
         "roofline": {"bound": "tensor", "achieved": round(gemm_tf, 1), "peak": round(fp8_burst, 1),
                      "unit": "TFLOP/s", "frac": round(gemm_tf / fp8_burst, 4),
                      "traffic": measured_traffic("gemm"),
-                     "kernel": "fp8_gemm_kernel (all 12 GEMM launches of a step, FLOP-weighted)",
+                     "kernel": "fp8_gemm_kernel (all GEMM launches of a step, FLOP-weighted: "
+                               + ("4 forward + 4 grouped dX+dW)" if stack.use_group_bwd() else "12 single GEMMs)"),
                      "peak_source": f"{peak_src}: 2 x bf16 burst {bf16_burst} TF/s (nominal fp8:bf16 = 2)",
                      "algorithmic_bytes_per_launch": round(g_bytes / n_g),
                      "flops_per_launch": round(g_flops / n_g),
@@ -837,6 +871,8 @@ def main():
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--one-stream", action="store_true", help="issue the whole step on one stream")
     ap.add_argument("--no-grouped", action="store_true", help="quantize every tensor with its own launch")
+    ap.add_argument("--no-group-bwd", action="store_true",
+                    help="run each linear's dX and dW as two GEMM launches (two streams) instead of one grouped launch")
     ap.add_argument("--split-k", type=int, default=0, help="force this many K splits in the GEMMs (0: library choice)")
     ap.add_argument("--dp-amax", action="store_true",
                     help="deferred ring folds + the ranks' amax all-reduce (MAX) and one fold per step")

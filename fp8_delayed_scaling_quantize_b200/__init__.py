@@ -57,6 +57,19 @@ class fp8_quantize_job(ctypes.Structure):
 
 assert ctypes.sizeof(fp8_quantize_job) == 56
 
+FP8_MM_MAX_GROUP = 4
+
+
+class fp8_mm_problem(ctypes.Structure):
+    """One problem of fp8_mm_grouped (pointers are device addresses)."""
+    _fields_ = [("a8", ctypes.c_void_p), ("b8", ctypes.c_void_p), ("sa", ctypes.c_void_p), ("sb", ctypes.c_void_p),
+                ("bias", ctypes.c_void_p), ("bias_scale", ctypes.c_void_p), ("out", ctypes.c_void_p),
+                ("M", ctypes.c_int64), ("N", ctypes.c_int64), ("K", ctypes.c_int64), ("fmt_a", ctypes.c_int32),
+                ("fmt_b", ctypes.c_int32), ("layout", ctypes.c_int32), ("bias_fmt", ctypes.c_int32)]
+
+
+assert ctypes.sizeof(fp8_mm_problem) == 96
+
 
 def _load():
     if not os.path.exists(LIB_PATH):
@@ -85,6 +98,7 @@ def _load():
         "fp8_mm_out8": (I, [P, I, P, I, P, P, I, I64, I64, I64, I64, I64, I64, I64, P, P, I, I, P, P, P, P, P]),
         "fp8_mm_splitk_static": (I, [P, I, P, I, P, P, I, I64, I64, I64, I64, I64, I64, I64, P, P, I, P,
                                      ctypes.c_int32, P]),
+        "fp8_mm_grouped": (I, [P, ctypes.c_int32, P]),
     }
     for name, (res, args) in sig.items():
         try:
@@ -207,6 +221,17 @@ def fp8_mm_out8(a8, fa, b8, fb, sa, sb, layout, M, N, K, batch, stride_a, stride
                                   int(M), int(N), int(K), int(batch), int(stride_a), int(stride_b), int(stride_c),
                                   _ptr(bias), _ptr(bias_scale), int(bias_fmt), int(out_fmt), _ptr(out_ring),
                                   _ptr(out8), _ptr(out_amax), _ptr(out_scale), _stream(stream)), "fp8_mm_out8")
+
+
+def fp8_mm_grouped(problems, stream=None):
+    """problems: sequence of (a8, fa, b8, fb, sa, sb, layout, M, N, K, bias,
+    bias_scale, bias_fmt, out), each as fp8_mm's arguments with batch 1."""
+    arr = (fp8_mm_problem * max(len(problems), 1))()
+    for i, (a8, fa, b8, fb, sa, sb, layout, M, N, K, bias, bias_scale, bias_fmt, out) in enumerate(problems):
+        arr[i] = fp8_mm_problem(_ptr(a8), _ptr(b8), _ptr(sa), _ptr(sb), _ptr(bias), _ptr(bias_scale), _ptr(out),
+                                int(M), int(N), int(K), int(fa), int(fb), int(layout), int(bias_fmt))
+    return _check(lib.fp8_mm_grouped(ctypes.cast(arr, ctypes.c_void_p), len(problems), _stream(stream)),
+                  "fp8_mm_grouped")
 
 
 def fp8_mm_workspace_size(M, N, K, batch, layout, split_k):

@@ -41,7 +41,9 @@
 
 #include <cuda_fp16.h>
 
+#include <algorithm>
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 #include "sm100.cuh"
@@ -86,6 +88,50 @@ struct GemmParams {
     float* out_scale;
     float* out_amax;
 };
+
+// Grouped launch (fp8_mm_grouped): several independent problems share one
+// persistent grid. Work units [unit_end of the previous problem, unit_end)
+// are the tiles of problem i; each role looks its unit's problem up here.
+constexpr int kMaxGroup = FP8_MM_MAX_GROUP;
+struct GroupProblem {
+    CUtensorMap ta, tb, tc;  // operand maps and the output's store map
+    int M, N, k_blocks, m_tiles, n_tiles, unit_end;
+    int a_mn, b_mn;
+    uint32_t idesc;
+    int bias_kind, bias_fmt, tma_store, vec_store;
+    const float* sa;
+    const float* sb;
+    const void* bias;
+    const float* bias_scale;
+    uint16_t* out;
+};
+template <bool GROUP>
+struct GroupTab {};  // single-problem launches carry no table
+template <>
+struct GroupTab<true> {
+    GroupProblem q[kMaxGroup];
+    int count;
+};
+
+// The i-th work unit of a CTA whose first unit is unit0, the persistent grid
+// holding unit_step CTAs (pairs). A grouped launch walks its rounds in
+// alternating directions: CTA c takes unit c of the first round, unit
+// step-1-c of the second, and so on. Its units come longest K first, so the
+// CTAs that drew the short tiles of one round take the first units of the
+// next, and no CTA stacks a second tile on a long one while others idle.
+template <bool GROUP>
+__device__ __forceinline__ int unit_of(int i, int unit0, int unit_step) {
+    return i * unit_step + ((GROUP && (i & 1)) ? unit_step - 1 - unit0 : unit0);
+}
+
+// The problem that work unit u of a grouped launch belongs to, and the
+// unit's tile index within it.
+__device__ __forceinline__ const GroupProblem& group_problem(const GroupTab<true>& g, int u, int& t) {
+    int i = 0;
+    while (i + 1 < g.count && u >= g.q[i].unit_end) ++i;
+    t = i == 0 ? u : u - g.q[i - 1].unit_end;
+    return g.q[i];
+}
 
 // Wait for phase `parity` of the mbarrier at `bar`, giving up after
 // `limit_ns`: then the library's device error word is set and false returned.
@@ -244,12 +290,19 @@ __device__ __forceinline__ bool epilogue_bar_or(bool v) {
 // Epilogue: 4 warps, one per TMEM lane quarter. Every 32 columns of the tile
 // become a 128 x 32 bf16 tile in shared memory that one thread writes with a
 // single TMA store (8 stores for a 128 x 256 tile).
-template <int BN, bool A_MN, bool B_MN, int STAGES, bool HAS_BIAS, int CTAS, bool SPLIT, bool SWAP, bool OUT8>
+//
+// GROUP: the units are the tiles of up to kMaxGroup problems (one SM per
+// tile, no split, no batches); operand majors, maps, scales, bias and output
+// come from the group table per unit, A_MN / B_MN only give the defaults.
+template <int BN, bool A_MN, bool B_MN, int STAGES, bool HAS_BIAS, int CTAS, bool SPLIT, bool SWAP, bool OUT8,
+          bool GROUP = false>
 __global__ void __maxnreg__(168)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                const __grid_constant__ CUtensorMap tm_c, const GemmParams p) {
+                const __grid_constant__ CUtensorMap tm_c, const GemmParams p,
+                const __grid_constant__ GroupTab<GROUP> grp) {
     using L = Smem<BN, STAGES, CTAS>;
     static_assert(!(B_MN && CTAS == 2 && BN != 256), "MN-major B halves must be whole 128-byte atoms");
+    static_assert(!GROUP || (CTAS == 1 && !SPLIT && !SWAP && !OUT8), "grouped launches use plain one-SM tiles");
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t s_base = smem_addr(smem);
@@ -278,8 +331,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     const TileWalk walk = {pin(p.m_tiles), pin(p.n_tiles), pin(p.group_m)};
     const int a_bcast = pin(p.a_bcast), b_bcast = pin(p.b_bcast);
     const uint32_t idesc = pin(p.idesc);
-    const int M = pin(p.M), N = pin(p.N);
-    const int tma_store = pin(p.tma_store), vec_store = pin(p.vec_store);
+    int M = pin(p.M), N = pin(p.N);  // per unit in a grouped launch
+    int tma_store = pin(p.tma_store), vec_store = pin(p.vec_store);
 
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -291,9 +344,17 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             mbar_init(bar_tempty + 8 * b, CTAS * kEpiThreads);
         }
         fence_mbar_init();
-        tma_prefetch(&tm_a);
-        tma_prefetch(&tm_b);
-        if (tma_store) tma_prefetch(&tm_c);
+        if constexpr (GROUP) {
+            for (int i = 0; i < grp.count; ++i) {
+                tma_prefetch(&grp.q[i].ta);
+                tma_prefetch(&grp.q[i].tb);
+                if (grp.q[i].tma_store) tma_prefetch(&grp.q[i].tc);
+            }
+        } else {
+            tma_prefetch(&tm_a);
+            tma_prefetch(&tm_b);
+            if (tma_store) tma_prefetch(&tm_c);
+        }
     }
     if (warp == 1) {
         tmem_alloc<CTAS>(smem_addr(tmem_slot), L::kTmemCols);
@@ -315,12 +376,26 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int u = unit0; u < total_units && ok; u += unit_step) {
-                const int t = u / split;
-                const int kb0 = (u - t * split) * kb_per;
-                const int kb1 = min(k_blocks, kb0 + kb_per);
+            for (int i = 0, u = unit0; u < total_units && ok; u = unit_of<GROUP>(++i, unit0, unit_step)) {
+                int t = u / split;
+                const CUtensorMap* map_a = &tm_a;
+                const CUtensorMap* map_b = &tm_b;
+                bool a_mn = A_MN, b_mn = B_MN;
+                TileWalk w = walk;
+                int kbs = k_blocks;
+                if constexpr (GROUP) {
+                    const GroupProblem& q = group_problem(grp, u, t);
+                    map_a = &q.ta;
+                    map_b = &q.tb;
+                    a_mn = q.a_mn;
+                    b_mn = q.b_mn;
+                    w = {q.m_tiles, q.n_tiles, walk.group_m};
+                    kbs = q.k_blocks;
+                }
+                const int kb0 = GROUP ? 0 : (u - t * split) * kb_per;
+                const int kb1 = GROUP ? kbs : min(k_blocks, kb0 + kb_per);
                 int mb, nb, b;
-                tile_coords(t, walk, mb, nb, b);
+                tile_coords(t, w, mb, nb, b);
                 const int ba = a_bcast ? 0 : b;
                 const int bb = b_bcast ? 0 : b;
                 const int m0 = mb * BM * CTAS + int(rank) * BM;
@@ -332,14 +407,14 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                     const uint32_t da = s_a + stage * L::kABytes;
                     const uint32_t db = s_b + stage * L::kBBytes;
                     if (CTAS == 1) {
-                        if (A_MN) tma_load_3d(da, &tm_a, full, m0, kb * BK, ba);
-                        else      tma_load_3d(da, &tm_a, full, kb * BK, m0, ba);
-                        if (B_MN) {
+                        if (a_mn) tma_load_3d(da, map_a, full, m0, kb * BK, ba);
+                        else      tma_load_3d(da, map_a, full, kb * BK, m0, ba);
+                        if (b_mn) {
 #pragma unroll
                             for (int h = 0; h < BN / 128; ++h)
-                                tma_load_3d(db + h * 128 * BK, &tm_b, full, n0 + h * 128, kb * BK, bb);
+                                tma_load_3d(db + h * 128 * BK, map_b, full, n0 + h * 128, kb * BK, bb);
                         } else {
-                            tma_load_3d(db, &tm_b, full, kb * BK, n0, bb);
+                            tma_load_3d(db, map_b, full, kb * BK, n0, bb);
                         }
                     } else {
                         const uint32_t lfull = map_to_rank(full, 0);  // the leader's barrier
@@ -364,10 +439,20 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             uint32_t phase = 0;
             int it = 0;
             bool ok = true;
-            for (int u = unit0; u < total_units && ok; u += unit_step, ++it) {
-                const int t = u / split;
-                const int kb0 = (u - t * split) * kb_per;
-                const int kb1 = min(k_blocks, kb0 + kb_per);
+            for (int u = unit0; u < total_units && ok; u = unit_of<GROUP>(++it, unit0, unit_step)) {
+                int t = u / split;
+                bool a_mn = A_MN, b_mn = B_MN;
+                uint32_t id = idesc;
+                int kbs = k_blocks;
+                if constexpr (GROUP) {
+                    const GroupProblem& q = group_problem(grp, u, t);
+                    a_mn = q.a_mn;
+                    b_mn = q.b_mn;
+                    id = q.idesc;
+                    kbs = q.k_blocks;
+                }
+                const int kb0 = GROUP ? 0 : (u - t * split) * kb_per;
+                const int kb1 = GROUP ? kbs : min(k_blocks, kb0 + kb_per);
                 const int buf = it & 1;
                 const uint32_t acc_phase = (it >> 1) & 1;
                 if (!wait_bounded(bar_tempty + 8 * buf, acc_phase ^ 1)) break;
@@ -382,11 +467,11 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                     for (int j = 0; j < BK / 32; ++j) {
                         // K-major: the 32-byte K step moves inside the swizzle atom;
                         // MN-major: it skips 32 rows of 128 bytes (4 atoms).
-                        const uint64_t adesc = A_MN ? smem_desc_sw128(da + j * 32 * 128, 128 * BK, 1024)
+                        const uint64_t adesc = a_mn ? smem_desc_sw128(da + j * 32 * 128, 128 * BK, 1024)
                                                     : smem_desc_sw128(da + j * 32, 16, 1024);
-                        const uint64_t bdesc = B_MN ? smem_desc_sw128(db + j * 32 * 128, 128 * BK, 1024)
+                        const uint64_t bdesc = b_mn ? smem_desc_sw128(db + j * 32 * 128, 128 * BK, 1024)
                                                     : smem_desc_sw128(db + j * 32, 16, 1024);
-                        mma_f8f6f4<CTAS>(d_tmem, adesc, bdesc, idesc, kb != kb0 || j != 0);
+                        mma_f8f6f4<CTAS>(d_tmem, adesc, bdesc, id, kb != kb0 || j != 0);
                     }
                     // release the stage (in both CTAs of a pair)
                     if (CTAS == 1) mma_commit(bar_empty + 8 * stage);
@@ -405,8 +490,12 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         const bool store_lead = etid == 0;  // issues the TMA stores
         const uint32_t stg0 = s_base + L::kStgOffset;
         int n_st = 0;  // TMA stores issued so far (they alternate between the two staging tiles)
-        const float inv = (1.0f / __ldg(p.sa)) * (1.0f / __ldg(p.sb));
-        const float bscale = (HAS_BIAS && p.bias_kind == 2) ? __ldg(p.bias_scale) : 1.0f;
+        float inv = (1.0f / __ldg(p.sa)) * (1.0f / __ldg(p.sb));
+        int bias_kind = p.bias_kind, bias_fmt = p.bias_fmt;
+        const void* bias_ptr = p.bias;
+        float bscale = (HAS_BIAS && bias_kind == 2) ? __ldg(p.bias_scale) : 1.0f;
+        uint16_t* out_base = p.out;
+        const CUtensorMap* map_c = &tm_c;
         // FP8 output: the ring's scale before this call (every CTA reads it
         // before any CTA can fold: the fold waits for all CTAs' tickets)
         float s_out = 1.0f, m_out = 0.0f;
@@ -416,11 +505,27 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         }
         bool failed = false;
         int it = 0;
-        for (int u = unit0; u < total_units; u += unit_step, ++it) {
-            const int t = u / split;
+        for (int u = unit0; u < total_units; u = unit_of<GROUP>(++it, unit0, unit_step)) {
+            int t = u / split;
             const int split_id = u - t * split;
+            TileWalk w = walk;
+            if constexpr (GROUP) {
+                const GroupProblem& q = group_problem(grp, u, t);
+                w = {q.m_tiles, q.n_tiles, walk.group_m};
+                M = q.M;
+                N = q.N;
+                tma_store = q.tma_store;
+                vec_store = q.vec_store;
+                map_c = &q.tc;
+                out_base = q.out;
+                bias_kind = q.bias_kind;
+                bias_fmt = q.bias_fmt;
+                bias_ptr = q.bias;
+                inv = (1.0f / __ldg(q.sa)) * (1.0f / __ldg(q.sb));
+                bscale = (HAS_BIAS && bias_kind == 2) ? __ldg(q.bias_scale) : 1.0f;
+            }
             int mb, nb, b;
-            tile_coords(t, walk, mb, nb, b);
+            tile_coords(t, w, mb, nb, b);
             const int buf = it & 1;
             const uint32_t acc_phase = (it >> 1) & 1;
             const int m0 = mb * BM * CTAS + int(rank) * BM;  // this CTA's first output row
@@ -430,11 +535,11 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                 for (int j = etid; j < BN; j += kEpiThreads) {
                     const int col = nb * BN + j;
                     float v = 0.0f;
-                    if (col < N) {
-                        if (p.bias_kind == 1) {
-                            v = __uint_as_float(uint32_t(__ldg(static_cast<const uint16_t*>(p.bias) + col)) << 16);
+                    if (col < N && bias_kind != 0) {  // a grouped launch may mix problems with and without bias
+                        if (bias_kind == 1) {
+                            v = __uint_as_float(uint32_t(__ldg(static_cast<const uint16_t*>(bias_ptr) + col)) << 16);
                         } else {
-                            v = __fdiv_rn(fp8_to_f32(__ldg(static_cast<const uint8_t*>(p.bias) + col), p.bias_fmt),
+                            v = __fdiv_rn(fp8_to_f32(__ldg(static_cast<const uint8_t*>(bias_ptr) + col), bias_fmt),
                                           bscale);
                         }
                     }
@@ -498,14 +603,14 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             // of C (the kernel's M is C's N), its accumulator columns are C's rows
             float bias_row = 0.0f;
             if (SWAP && HAS_BIAS && row < M) {
-                if (p.bias_kind == 1)
-                    bias_row = __uint_as_float(uint32_t(__ldg(static_cast<const uint16_t*>(p.bias) + row)) << 16);
+                if (bias_kind == 1)
+                    bias_row = __uint_as_float(uint32_t(__ldg(static_cast<const uint16_t*>(bias_ptr) + row)) << 16);
                 else
-                    bias_row = __fdiv_rn(fp8_to_f32(__ldg(static_cast<const uint8_t*>(p.bias) + row), p.bias_fmt),
+                    bias_row = __fdiv_rn(fp8_to_f32(__ldg(static_cast<const uint8_t*>(bias_ptr) + row), bias_fmt),
                                          bscale);
             }
-            uint16_t* orow = SWAP ? p.out + int64_t(b) * p.stride_c + row
-                                  : p.out + int64_t(b) * p.stride_c + int64_t(row) * N;
+            uint16_t* orow = SWAP ? out_base + int64_t(b) * p.stride_c + row
+                                  : out_base + int64_t(b) * p.stride_c + int64_t(row) * N;
 #pragma unroll 1
             for (int c = 0; c < BN / CW; ++c) {
                 const int col0 = nb * BN + c * CW;
@@ -573,7 +678,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                                        (cvt_fp8x2(p.out_fmt, __fmul_rn(y[4 * j + 2], s_out),
                                                   __fmul_rn(y[4 * j + 3], s_out)) << 16);
                             }
-                            uint8_t* dst = reinterpret_cast<uint8_t*>(p.out) + int64_t(b) * p.stride_c +
+                            uint8_t* dst = reinterpret_cast<uint8_t*>(out_base) + int64_t(b) * p.stride_c +
                                            int64_t(row) * N + col0;
                             if (vec_store && col0 + 32 <= N) {
                                 reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
@@ -607,7 +712,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                         if (store_lead) bulk_wait_read<0>();
                         epilogue_bar();
                         if (store_lead) {
-                            tma_store_3d(&tm_c, stg, col0, m0, b);
+                            tma_store_3d(map_c, stg, col0, m0, b);
                             bulk_commit();
                         }
                         ++n_st;
@@ -642,7 +747,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         // the staging tiles must outlive the stores that read them; the global
         // writes themselves complete with the grid (a dependent kernel's
         // griddepcontrol.wait and stream order both see them)
-        if (tma_store && store_lead) bulk_wait_read<0>();
+        if ((GROUP || tma_store) && store_lead) bulk_wait_read<0>();
         if constexpr (OUT8) {
             // the CTA's amax of the output: one atomicMax, then a ticket; the
             // CTA holding the last ticket folds it into the output's ring
@@ -779,7 +884,7 @@ fp8_status launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
     p.total_units = int(work);
     const int64_t units_max = sm_count() / CTAS;
     const int units = int(work < units_max ? work : units_max);
-    return launch_pdl(kern, units * CTAS, kThreads, L::kAlloc, st, CTAS, ta, tb, tc, p);
+    return launch_pdl(kern, units * CTAS, kThreads, L::kAlloc, st, CTAS, ta, tb, tc, p, GroupTab<false>{});
 }
 
 template <int BN, bool A_MN, bool B_MN, int STAGES, int CTAS, bool SWAP = false, bool OUT8 = false>
@@ -1069,6 +1174,138 @@ fp8_status mm_impl(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8, fp8_fmt fb,
     }
 }
 
+
+// ------------------------------------------------------- grouped launch ---
+
+template <int BN, int STAGES, bool HAS_BIAS>
+fp8_status launch_group(const GroupTab<true>& g, int total_units, cudaStream_t st) {
+    using L = Smem<BN, STAGES, 1>;
+    auto kern = fp8_gemm_kernel<BN, false, false, STAGES, HAS_BIAS, 1, false, false, false, true>;
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8_ERR_CUDA;
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) != cudaSuccess)
+            return FP8_ERR_CUDA;
+        attr_set[dev] = true;
+    }
+    // the kernel-wide parameters a grouped launch still reads: the unit
+    // count, the walk's group height, and valid scale pointers for the
+    // epilogue's set-up (every unit reloads its own problem's scales)
+    GemmParams p = {};
+    p.total_units = total_units;
+    p.total_tiles = total_units;
+    p.split = 1;
+    p.group_m = 16;
+    p.a_bcast = 1;
+    p.b_bcast = 1;
+    p.sa = g.q[0].sa;
+    p.sb = g.q[0].sb;
+    const int units = total_units < sm_count() ? total_units : sm_count();
+    const CUtensorMap none = {};
+    return launch_pdl(kern, units, kThreads, L::kAlloc, st, 1, none, none, none, p, g);
+}
+
+// Tile width of a grouped launch: the persistent grid hands out the units in
+// rounds of `grid`, alternating direction (unit_of), so the launch lasts as
+// long as its busiest CTA; this is that CTA's k-blocks (times the per-k-block
+// cost of the tile width) plus one exposed epilogue, the same cost model as a
+// single problem's choice.
+inline int choose_group_bn(const int64_t* M, const int64_t* N, const int64_t* kb, int count, int64_t sms) {
+    int best_bn = 256;
+    double best = 1e30;
+    for (int bn : {256, 128}) {
+        const double t_k = bn == 256 ? 0.48 : 0.40, t_epi = bn == 256 ? 2.0 : 1.0;
+        int64_t total = 0;
+        for (int i = 0; i < count; ++i) total += ((M[i] + BM - 1) / BM) * ((N[i] + bn - 1) / bn);
+        const int64_t grid = total < sms ? total : sms;
+        std::vector<int64_t> load(size_t(grid), 0);
+        int64_t u = 0;
+        for (int i = 0; i < count; ++i) {
+            const int64_t tiles = ((M[i] + BM - 1) / BM) * ((N[i] + bn - 1) / bn);
+            for (int64_t k = 0; k < tiles; ++k, ++u) {
+                const int64_t round = u / grid, pos = u - round * grid;
+                load[size_t((round & 1) ? grid - 1 - pos : pos)] += kb[i];
+            }
+        }
+        const int64_t worst = *std::max_element(load.begin(), load.end());
+        const double c = double(worst) * t_k + t_epi;
+        if (c < best) { best = c; best_bn = bn; }
+    }
+    return best_bn;
+}
+
+fp8_status mm_grouped_impl(const fp8_mm_problem* probs, int32_t count, void* stream) {
+    if (!probs || count < 1 || count > kMaxGroup) return FP8_ERR_INVALID_ARG;
+    for (int i = 0; i < count; ++i) {
+        const fp8_mm_problem& q = probs[i];
+        if (!valid_fmt(q.fmt_a) || !valid_fmt(q.fmt_b)) return FP8_ERR_INVALID_ARG;
+        if (q.layout != FP8_NT && q.layout != FP8_NN && q.layout != FP8_TN) return FP8_ERR_INVALID_ARG;
+        if (!q.a8 || !q.b8 || !q.sa || !q.sb || !q.out) return FP8_ERR_INVALID_ARG;
+        if (q.M < 1 || q.N < 1 || q.K < 1) return FP8_ERR_INVALID_ARG;
+        if (q.bias_scale && !q.bias) return FP8_ERR_INVALID_ARG;
+        if (q.bias && q.bias_scale && !valid_fmt(q.bias_fmt)) return FP8_ERR_INVALID_ARG;
+        if (q.M >= (int64_t(1) << 31) || q.N >= (int64_t(1) << 31) || q.K >= (int64_t(1) << 31))
+            return FP8_ERR_UNSUPPORTED;
+        const bool a_mn = q.layout == FP8_TN, b_mn = q.layout != FP8_NT;
+        if ((a_mn ? q.M : q.K) % 16 != 0 || (b_mn ? q.N : q.K) % 16 != 0) return FP8_ERR_ALIGNMENT;
+        if (!aligned(q.a8, 16) || !aligned(q.b8, 16)) return FP8_ERR_ALIGNMENT;
+        if (!aligned(q.out, 4) || !aligned(q.sa, 4) || !aligned(q.sb, 4)) return FP8_ERR_ALIGNMENT;
+        if (q.bias && !q.bias_scale && !aligned(q.bias, 2)) return FP8_ERR_ALIGNMENT;
+    }
+    // longest K first: the first wave of the persistent grid starts the
+    // tiles that take longest, the shorter ones fill in behind them
+    int order[kMaxGroup];
+    for (int i = 0; i < count; ++i) order[i] = i;
+    std::stable_sort(order, order + count, [&](int x, int y) { return probs[x].K > probs[y].K; });
+    int64_t M[kMaxGroup], N[kMaxGroup], kb[kMaxGroup];
+    for (int i = 0; i < count; ++i) {
+        M[i] = probs[order[i]].M;
+        N[i] = probs[order[i]].N;
+        kb[i] = (probs[order[i]].K + BK - 1) / BK;
+    }
+    const int bn = choose_group_bn(M, N, kb, count, sm_count());
+    GroupTab<true> g = {};
+    g.count = count;
+    int64_t units = 0;
+    bool any_bias = false;
+    for (int i = 0; i < count; ++i) {
+        const fp8_mm_problem& q = probs[order[i]];
+        GroupProblem& d = g.q[i];
+        const bool a_mn = q.layout == FP8_TN, b_mn = q.layout != FP8_NT;
+        const bool ok = (a_mn ? make_map(&d.ta, q.a8, q.M, q.K, 1, 0, 128, BK)
+                              : make_map(&d.ta, q.a8, q.K, q.M, 1, 0, BK, BM)) &&
+                        (b_mn ? make_map(&d.tb, q.b8, q.N, q.K, 1, 0, 128, BK)
+                              : make_map(&d.tb, q.b8, q.K, q.N, 1, 0, BK, uint32_t(bn)));
+        if (!ok) return FP8_ERR_CUDA;
+        d.M = int(q.M);
+        d.N = int(q.N);
+        d.k_blocks = int(kb[i]);
+        d.m_tiles = int((q.M + BM - 1) / BM);
+        d.n_tiles = int((q.N + bn - 1) / bn);
+        units += int64_t(d.m_tiles) * d.n_tiles;
+        if (units >= (int64_t(1) << 31)) return FP8_ERR_UNSUPPORTED;
+        d.unit_end = int(units);
+        d.a_mn = a_mn;
+        d.b_mn = b_mn;
+        d.idesc = sm100::instr_desc_f8(q.fmt_a, q.fmt_b, a_mn, b_mn, BM, bn);
+        d.bias_kind = q.bias ? (q.bias_scale ? 2 : 1) : 0;
+        d.bias_fmt = q.bias_fmt;
+        any_bias = any_bias || q.bias;
+        d.vec_store = (q.N % 8 == 0) && aligned(q.out, 16);
+        d.tma_store = d.vec_store;
+        if (d.tma_store && !make_out_map(&d.tc, q.out, q.N, q.M, 1, 0)) return FP8_ERR_CUDA;
+        d.sa = q.sa;
+        d.sb = q.sb;
+        d.bias = q.bias;
+        d.bias_scale = q.bias_scale;
+        d.out = static_cast<uint16_t*>(q.out);
+    }
+    cudaStream_t st = as_stream(stream);
+    if (bn == 256)
+        return any_bias ? launch_group<256, 4, true>(g, int(units), st) : launch_group<256, 4, false>(g, int(units), st);
+    return any_bias ? launch_group<128, 6, true>(g, int(units), st) : launch_group<128, 6, false>(g, int(units), st);
+}
 }  // namespace
 }  // namespace fp8lite
 
@@ -1151,4 +1388,8 @@ extern "C" fp8_status fp8_selftest_wait_timeout(uint32_t limit_us, void* stream)
     if (limit_us == 0 || limit_us > 1000000u) return FP8_ERR_INVALID_ARG;
     selftest_wait_kernel<<<1, 1, 0, as_stream(stream)>>>(uint64_t(limit_us) * 1000ull);
     return launch_status();
+}
+
+extern "C" fp8_status fp8_mm_grouped(const fp8_mm_problem* problems, int32_t count, void* stream) {
+    return mm_grouped_impl(problems, count, stream);
 }

@@ -26,7 +26,7 @@
 extern "C" {
 #endif
 
-#define FP8LITE_ABI_VERSION 2
+#define FP8LITE_ABI_VERSION 3
 
 /* Exported entry points (the library is built with hidden visibility). */
 #if defined(__GNUC__)
@@ -352,6 +352,38 @@ FP8LITE_API fp8_status fp8_mm_splitk_static(const uint8_t* a8, fp8_fmt fa, const
                   int64_t stride_a, int64_t stride_b, int64_t stride_c,
                   const void* bias, const float* bias_scale, fp8_fmt bias_fmt,
                   void* out, int32_t split_k, void* stream);
+
+/* Several independent fp8_mm problems in ONE launch: their output tiles
+ * share one persistent grid, one prologue and one tail. Made for the
+ * backward pass of a linear layer, whose dX (NN) and dW (TN) GEMMs both read
+ * the gradient's codes and nothing of each other [test_fp8_mma.py@cebdd45d,
+ * the dX / dW layout cases]. Each problem computes exactly what fp8_mm
+ * computes with batch 1 (out = bf16_rne(acc/(sa*sb) + bias_j), fp32
+ * accumulation over K in the same k-block order), so its output equals
+ * fp8_mm's bit for bit.
+ *
+ * problems  HOST array of `count` descriptions (read during the call only)
+ * count     1 .. FP8_MM_MAX_GROUP
+ * Per problem, the fields mean what fp8_mm's arguments of the same name mean,
+ * with batch = 1 and out a contiguous row-major bf16 [M, N]. The outputs
+ * must not overlap each other or any operand.
+ * Errors: as fp8_mm for any one problem (the first failing check decides),
+ *         FP8_ERR_INVALID_ARG for a NULL array or count out of range. */
+#define FP8_MM_MAX_GROUP 4
+typedef struct fp8_mm_problem {
+    const uint8_t* a8;
+    const uint8_t* b8;
+    const float* sa;
+    const float* sb;
+    const void* bias;        /* NULL, bf16[N], or FP8 codes[N] of bias_fmt */
+    const float* bias_scale; /* NULL (bf16 bias) or device float (FP8 bias) */
+    void* out;               /* device bf16[M*N], 4-byte aligned */
+    int64_t M, N, K;
+    int32_t fmt_a, fmt_b;    /* fp8_fmt values */
+    int32_t layout;          /* fp8_layout value */
+    int32_t bias_fmt;        /* fp8_fmt value, read only for an FP8 bias */
+} fp8_mm_problem;
+FP8LITE_API fp8_status fp8_mm_grouped(const fp8_mm_problem* problems, int32_t count, void* stream);
 
 /* Synchronises the current device, then reads and clears the library's
  * device error word: FP8_ERR_DEVICE_TIMEOUT if a GEMM thread block gave up a

@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(fp8):
 
 
 def test_abi_version_and_status_strings(fp8):
-    assert fp8.fp8_abi_version() == 2
+    assert fp8.fp8_abi_version() == 3
     for code, name in [(0, "FP8_OK"), (1, "FP8_ERR_INVALID_ARG"), (2, "FP8_ERR_ALIGNMENT"),
                        (3, "FP8_ERR_UNSUPPORTED"), (4, "FP8_ERR_CUDA"), (5, "FP8_ERR_DEVICE_TIMEOUT")]:
         assert fp8.status_string(code) == name
@@ -206,3 +206,32 @@ def test_mm_out8_validation(fp8):
     assert st(scale=None) == fp8.FP8_ERR_INVALID_ARG
     assert st(out8=None) == fp8.FP8_ERR_INVALID_ARG
     assert st(ring=S + 2) == fp8.FP8_ERR_ALIGNMENT
+
+
+def test_mm_grouped_validation(fp8):
+    def prob(**kw):
+        d = dict(a8=A, b8=A, sa=S, sb=S, bias=None, bias_scale=None, out=A + 262144, M=128, N=128, K=128,
+                 fmt_a=0, fmt_b=0, layout=0, bias_fmt=0)
+        d.update(kw)
+        return fp8.fp8_mm_problem(**d)
+
+    def st(probs, count=None):
+        arr = (fp8.fp8_mm_problem * max(len(probs), 1))(*probs)
+        return fp8.raw_status("fp8_mm_grouped", ctypes.cast(arr, ctypes.c_void_p),
+                              len(probs) if count is None else count, None)
+    E, AL, U = fp8.FP8_ERR_INVALID_ARG, fp8.FP8_ERR_ALIGNMENT, fp8.FP8_ERR_UNSUPPORTED
+    assert fp8.raw_status("fp8_mm_grouped", None, 1, None) == E
+    assert st([prob()], count=0) == E
+    assert st([prob()] * (fp8.FP8_MM_MAX_GROUP + 1)) == E
+    assert st([prob(), prob(fmt_a=3)]) == E           # the second problem decides
+    assert st([prob(layout=3)]) == E
+    assert st([prob(out=None)]) == E and st([prob(sb=None)]) == E
+    assert st([prob(), prob(M=0)]) == E and st([prob(K=0)]) == E
+    assert st([prob(bias_scale=S + 8)]) == E           # a scale without a bias
+    assert st([prob(bias=A, bias_scale=S + 8, bias_fmt=7)]) == E
+    assert st([prob(N=1 << 31)]) == U
+    assert st([prob(K=100)]) == AL                     # TMA row pitches, as fp8_mm
+    assert st([prob(layout=1, N=100)]) == AL
+    assert st([prob(layout=2, M=100)]) == AL
+    assert st([prob(), prob(b8=A + 8)]) == AL
+    assert st([prob(out=A + 2)]) == AL
