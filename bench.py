@@ -800,6 +800,23 @@ def run_kernel(args):
         call = lambda i: fp8.fp8_mm_ws(sets[i % 2][0], E4M3, sets[i % 2][1], E4M3, sa, sa, layout, M, N, K, 1, 0, 0,
                                        0, None, None, 0, out, ws, args.split_k if need else 0, stream=st)
         units = 2.0 * M * N * K
+    elif args.kernel == "bwd_pair":
+        # a linear's backward as the step runs it: dX = g W (NN) and
+        # dW = g^T x (TN) in one grouped launch; --shape T x d_in x d_out
+        T, d_in, d_out = (int(v) for v in args.shape.split("x"))
+        sets = []
+        for i in range(2):
+            g8 = W.fp8_codes((T * d_out,), E5M2, 9600 + i).cuda()
+            w8 = W.fp8_codes((d_out * d_in,), E4M3, 9700 + i).cuda()
+            x8 = W.fp8_codes((T * d_in,), E4M3, 9800 + i).cuda()
+            sets.append((g8, w8, x8))
+        sa = torch.ones(1, device="cuda")
+        dx = torch.empty(T * d_in, dtype=torch.bfloat16, device="cuda")
+        dw = torch.empty(d_out * d_in, dtype=torch.bfloat16, device="cuda")
+        call = lambda i: fp8.fp8_mm_grouped(
+            [(sets[i % 2][0], E5M2, sets[i % 2][1], E4M3, sa, sa, NN, T, d_in, d_out, None, None, 0, dx),
+             (sets[i % 2][0], E5M2, sets[i % 2][2], E4M3, sa, sa, TN, d_out, d_in, T, None, None, 0, dw)], stream=st)
+        units = 2.0 * 2 * T * d_in * d_out
     elif args.kernel == "quantize_2d":
         # both orientations of a bf16 [rows, cols] tensor from one pass, delayed
         rows, cols = (int(v) for v in args.shape.split("x"))
@@ -848,11 +865,12 @@ def run_kernel(args):
         e1.record(st)
     torch.cuda.synchronize()
     us = e0.elapsed_time(e1) * 1e3 / reps
-    if args.kernel in ("gemm", "cublaslt"):
+    if args.kernel in ("gemm", "cublaslt", "bwd_pair"):
         ach = units / (us * 1e-6) / 1e12
         peak = 2 * bf16_burst
         print(json.dumps({"kernel": args.kernel, "shape": args.shape,
-                          "layout": args.layout if args.kernel == "gemm" else "NT", "us": round(us, 2),
+                          "layout": {"gemm": args.layout, "cublaslt": "NT", "bwd_pair": "NN + TN"}[args.kernel],
+                          "us": round(us, 2),
                           "tflops": round(ach, 1), "frac_fp8_peak": round(ach / peak, 4), "peak": peak,
                           "peak_source": src}))
     else:
@@ -881,7 +899,7 @@ def main():
     ap.add_argument("--no-compare", action="store_true", help="skip the bf16 / autograd comparison")
     ap.add_argument("--breakdown-reps", type=int, default=20)
     ap.add_argument("--e2e-steps", type=int, default=10)
-    ap.add_argument("--kernel", choices=["gemm", "quantize", "quantize_many", "quantize_2d", "cublaslt"],
+    ap.add_argument("--kernel", choices=["gemm", "bwd_pair", "quantize", "quantize_many", "quantize_2d", "cublaslt"],
                     help="single-kernel mode")
     ap.add_argument("--shape", default="8192x8192x8192", help="MxNxK for gemm, n for quantize")
     ap.add_argument("--layout", default="NT", choices=["NT", "NN", "TN"])
