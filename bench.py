@@ -15,7 +15,8 @@ value  = GEMM FLOPs of the step (154.6 GFLOP) / device step time, TFLOP/s,
          resident in HBM, rotating through 3 input sets (276 MB > 126 MB L2).
 e2e    = the same metric through the public API with HOST buffers: pinned
          host -> device copies of x, W, g and device -> host copies of y,
-         dX, dW inside the timed region, eager calls.
+         dX, dW inside the timed region, eager calls; the copies of
+         consecutive steps overlap (double buffers, one copy stream each way).
 roofline / roofline_quantize = the GEMM kernel and the quantize kernel,
          each timed per launch with CUDA events on the launching stream.
 cpu_baseline = the CPU oracle (numpy, fp64 GEMM) on one full step.
@@ -627,39 +628,67 @@ def compare_bf16(stack, fp8_ms, reps):
 
 def run_e2e(fp8, stack, stream, steps, world, side=None, grouped=True):
     """H2D of the step's inputs from pinned host memory, the step's calls, D2H of
-    the three GEMM outputs, per step; CUDA events around the whole loop."""
+    the three GEMM outputs, every step; CUDA events around the whole loop.
+
+    The copies are pipelined as a training input pipeline would be: inputs
+    and outputs are double-buffered on the device, host-to-device copies run
+    on one copy stream and device-to-host copies on another (PCIe is full
+    duplex), so step i's outputs leave while step i+1's inputs arrive. Every
+    step still moves all of its bytes both ways inside the timed region."""
     host_in = [{k: v.cpu().pin_memory() for k, v in t.items()} for t in stack.sets[0]]
-    host_out = [{k: torch.empty(L[k].numel(), dtype=torch.bfloat16).pin_memory() for k in ("y", "dx", "dw")}
-                for L in stack.lin]
+    outs = [[{k: L[k] for k in ("y", "dx", "dw")} for L in stack.lin],
+            [{k: torch.empty_like(L[k]) for k in ("y", "dx", "dw")} for L in stack.lin]]
+    host_out = [[{k: torch.empty(L[k].numel(), dtype=torch.bfloat16).pin_memory() for k in ("y", "dx", "dw")}
+                 for L in stack.lin] for _ in range(2)]
     h2d = sum(v.numel() * 2 for t in host_in for v in t.values())
-    d2h = sum(v.numel() * 2 for t in host_out for v in t.values())
+    d2h = sum(v.numel() * 2 for t in host_out[0] for v in t.values())
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = {k: [torch.cuda.Event(), torch.cuda.Event()] for k in ("in", "used", "out", "sent")}
+    for k in ("used", "sent"):
+        for e in ev[k]:
+            e.record(stream)
 
-    def one():
-        for li, t in enumerate(host_in):
-            for k, v in t.items():
-                stack.sets[0][li][k].copy_(v, non_blocking=True)
-        stack.step(0, stream, side, grouped)
-        for li, L in enumerate(stack.lin):
-            for k in ("y", "dx", "dw"):
-                host_out[li][k].copy_(L[k], non_blocking=True)
+    def one(i):
+        p = i % 2  # input set p and output buffers p
+        up.wait_event(ev["used"][p])          # step i-2 has finished reading set p
+        with torch.cuda.stream(up):
+            for li, t in enumerate(host_in):
+                for k, v in t.items():
+                    stack.sets[p][li][k].copy_(v, non_blocking=True)
+        ev["in"][p].record(up)
+        stream.wait_event(ev["in"][p])
+        stream.wait_event(ev["sent"][p])      # step i-2's outputs p have left
+        for L, o in zip(stack.lin, outs[p]):
+            L.update(o)
+        stack.step(p, stream, side, grouped)
+        ev["used"][p].record(stream)
+        down.wait_event(ev["used"][p])
+        with torch.cuda.stream(down):
+            for li, L in enumerate(outs[p]):
+                for k in ("y", "dx", "dw"):
+                    host_out[p][li][k].copy_(L[k], non_blocking=True)
+        ev["sent"][p].record(down)
 
-    with torch.cuda.stream(stream):
-        for _ in range(2):
-            one()
+    for i in range(2):
+        one(i)
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(steps):
-            one()
-        e1.record(stream)
+    e0.record(stream)
+    for i in range(steps):
+        one(i)
+    stream.wait_stream(up)
+    stream.wait_stream(down)
+    e1.record(stream)
     e1.synchronize()
     barrier(world)
+    for L, o in zip(stack.lin, outs[0]):
+        L.update(o)
     t_ms = max_over_ranks(e0.elapsed_time(e1), world)
     return {"value": weak_scaling_value(stack.flops, steps, world, t_ms), "unit": "TFLOP/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "ms_per_step": round(t_ms / steps, 3)}
+            "ms_per_step": round(t_ms / steps, 3),
+            "pipeline": "inputs and outputs double-buffered; H2D and D2H on two copy streams"}
 
 
 # ------------------------------------------------------- the CPU oracle -----
@@ -898,7 +927,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-compare", action="store_true", help="skip the bf16 / autograd comparison")
     ap.add_argument("--breakdown-reps", type=int, default=20)
-    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--kernel", choices=["gemm", "bwd_pair", "quantize", "quantize_many", "quantize_2d", "cublaslt"],
                     help="single-kernel mode")
     ap.add_argument("--shape", default="8192x8192x8192", help="MxNxK for gemm, n for quantize")

@@ -113,6 +113,18 @@ def test_grouped_many_tiles_unequal_k(g):
         p.check_same_as_fp8_mm(g, f"unequal k problem {i} vs fp8_mm")
 
 
+def test_grouped_three_layouts_ragged_mid_size(g):
+    """Three mid-size problems (several rounds of the persistent grid), ragged
+    M and N, every layout, both bias kinds."""
+    specs = [(NT, 1500, 1700, 512, E4M3, E4M3, 1), (NN, 1200, 1808, 256, E5M2, E4M3, 0),
+             (TN, 704, 912, 640, E5M2, E4M3, 2)]
+    probs = [Prob(*s[:6], seed=800 + 10 * i, bias_kind=s[6]) for i, s in enumerate(specs)]
+    _run(probs)
+    for i, p in enumerate(probs):
+        p.check_full(g, f"mid-size problem {i}")
+        p.check_same_as_fp8_mm(g, f"mid-size problem {i} vs fp8_mm")
+
+
 def _sample_idx(M, N, seed):
     rng = np.random.default_rng(seed)
     i = rng.integers(0, M, 2048)
