@@ -541,61 +541,68 @@ def run_ours(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
-def _graph_time(fn, stream, reps, warm=3):
-    """Capture fn() in a CUDA graph on `stream`; return ms per replay."""
+def _rotated_graph_time(make_fn, reps, warm=3):
+    """One CUDA graph per input set, replayed in rotation over the sets, as
+    the FP8 step is timed; ms per replay."""
+    st = torch.cuda.Stream()
+    fns = [make_fn(s) for s in range(N_SETS)]
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(side):
         for _ in range(warm):
-            fn()
+            for f in fns:
+                f()
     torch.cuda.current_stream().wait_stream(side)
     torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
-        fn()
+    graphs = []
+    for f in fns:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=st):
+            f()
+        graphs.append(g)
     torch.cuda.synchronize()
-    with torch.cuda.stream(stream):
-        for _ in range(warm):
-            g.replay()
+    with torch.cuda.stream(st):
+        for i in range(warm * N_SETS):
+            graphs[i % N_SETS].replay()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(reps):
-            g.replay()
-        e1.record(stream)
+        e0.record(st)
+        for i in range(reps):
+            graphs[i % N_SETS].replay()
+        e1.record(st)
     e1.synchronize()
     ms = e0.elapsed_time(e1) / reps
-    del g
+    graphs.clear()
     return ms
 
 
 def compare_bf16(stack, fp8_ms, reps):
-    """The same linear-stack training step as bf16 GEMMs on cuBLAS
-    (torch.matmul; forward, then dX and dW in reverse, dW on a second
-    stream), and the step through the autograd layer (Fp8Linear vs bf16
-    nn.Linear), each as a CUDA graph: the FP8-over-bf16 speed-up the
-    AstrAI commit logs report for their kernels."""
+    """The same linear-stack training step with bf16 GEMMs on cuBLAS
+    (torch.matmul: forward, then dX and dW in reverse, one stream, which
+    measured faster than putting dW on a second stream), and the step
+    through the autograd layer (Fp8Linear against bf16 nn.Linear). Each is
+    timed like the FP8 step: CUDA graphs over the same 3 rotating input sets
+    (the autograd modules keep one weight each, as in training). Context
+    for the FP8-over-bf16 speed-up the AstrAI commit logs report for their
+    kernels on L20."""
     out = {}
     T = W.TOKENS
-    ts = stack.sets[0]
     ys = [torch.empty(T, L["d_out"], dtype=torch.bfloat16, device="cuda") for L in stack.lin]
     dxs = [torch.empty(T, L["d_in"], dtype=torch.bfloat16, device="cuda") for L in stack.lin]
     dws = [torch.empty(L["d_out"], L["d_in"], dtype=torch.bfloat16, device="cuda") for L in stack.lin]
-    side = torch.cuda.Stream()
 
-    def bf16_step():
-        cur = torch.cuda.current_stream()
-        for li, t in enumerate(ts):
-            torch.matmul(t["x"], t["w"].t(), out=ys[li])
-        for li in reversed(range(len(ts))):
-            t = ts[li]
-            side.wait_stream(cur)
-            with torch.cuda.stream(side):
+    def bf16_step(s):
+        ts = stack.sets[s]
+
+        def fn():
+            for li, t in enumerate(ts):
+                torch.matmul(t["x"], t["w"].t(), out=ys[li])
+            for li in reversed(range(len(ts))):
+                t = ts[li]
+                torch.matmul(t["g"], t["w"], out=dxs[li])
                 torch.matmul(t["g"].t(), t["x"], out=dws[li])
-            torch.matmul(t["g"], t["w"], out=dxs[li])
-            cur.wait_stream(side)
+        return fn
 
-    st = torch.cuda.Stream()
-    bf16_ms = _graph_time(bf16_step, st, reps)
+    bf16_ms = _rotated_graph_time(bf16_step, reps)
     out["bf16_cublas_step_ms"] = round(bf16_ms, 4)
     out["fp8_over_bf16_step"] = round(bf16_ms / fp8_ms, 3)
 
@@ -605,21 +612,22 @@ def compare_bf16(stack, fp8_ms, reps):
         mods8 = [Fp8Linear(L["d_in"], L["d_out"], bias=False, device="cuda") for L in stack.lin]
         mods16 = [torch.nn.Linear(L["d_in"], L["d_out"], bias=False, device="cuda", dtype=torch.bfloat16)
                   for L in stack.lin]
-        xs = [t["x"].detach().clone().requires_grad_(True) for t in ts]
-        gs = [t["g"] for t in ts]
+        xs = [[t["x"].detach().clone().requires_grad_(True) for t in stack.sets[s]] for s in range(N_SETS)]
 
         def ag_step(mods):
-            def fn():
-                for m in mods:
-                    m.weight.grad = None
-                for x in xs:
-                    x.grad = None
-                ys_ = [m(x) for m, x in zip(mods, xs)]
-                torch.autograd.backward(ys_, gs)
-            return fn
+            def make(s):
+                def fn():
+                    for m in mods:
+                        m.weight.grad = None
+                    for x in xs[s]:
+                        x.grad = None
+                    ys_ = [m(x) for m, x in zip(mods, xs[s])]
+                    torch.autograd.backward(ys_, [t["g"] for t in stack.sets[s]])
+                return fn
+            return make
 
-        out["autograd_fp8_step_ms"] = round(_graph_time(ag_step(mods8), st, reps), 4)
-        out["autograd_bf16_step_ms"] = round(_graph_time(ag_step(mods16), st, reps), 4)
+        out["autograd_fp8_step_ms"] = round(_rotated_graph_time(ag_step(mods8), reps), 4)
+        out["autograd_bf16_step_ms"] = round(_rotated_graph_time(ag_step(mods16), reps), 4)
         out["autograd_fp8_over_bf16"] = round(out["autograd_bf16_step_ms"] / out["autograd_fp8_step_ms"], 3)
     except Exception as e:  # capture failures are reported, not hidden
         out["autograd_error"] = f"{type(e).__name__}: {e}"[:200]

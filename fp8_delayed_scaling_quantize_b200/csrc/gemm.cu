@@ -459,8 +459,11 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + buf * BN;
                 for (int kb = kb0; kb < kb1; ++kb) {
+                    // the stage's operands arrive through the async proxy and
+                    // complete on this barrier: the MMAs may read them without
+                    // a tcgen05 fence (that is needed only after the epilogue's
+                    // hand-back of the accumulator, above)
                     if (!wait_bounded(bar_full + 8 * stage, phase)) { ok = false; break; }
-                    tc_fence_after();
                     const uint32_t da = s_a + stage * L::kABytes;
                     const uint32_t db = s_b + stage * L::kBBytes;
 #pragma unroll

@@ -25,7 +25,7 @@ state_dict for checkpoint and resume.
 import torch
 
 from . import (FP8_E4M3, FP8_E5M2, FP8_NN, FP8_NT, FP8_RING_BYTES, FP8_TN, fp8_bias_grad, fp8_mm, fp8_mm_grouped,
-               fp8_quantize, fp8_ring_init)
+               fp8_quantize, fp8_quantize_many, fp8_ring_init)
 
 _RING_WORDS = FP8_RING_BYTES // 4
 
@@ -51,8 +51,14 @@ class Fp8LinearFunction(torch.autograd.Function):
         x2 = x.reshape(-1, K).contiguous()
         w = weight.contiguous()
         T = x2.shape[0]
-        x8, sx = _quantize(x2, T * K, FP8_E4M3, rings[0])
-        w8, sw = _quantize(w, N * K, FP8_E4M3, rings[1])
+        # x and W in one quantize launch (each with its own ring)
+        dev = x.device
+        x8 = torch.empty(T * K, dtype=torch.uint8, device=dev)
+        w8 = torch.empty(N * K, dtype=torch.uint8, device=dev)
+        stats = torch.empty(4, dtype=torch.float32, device=dev)  # amax x, amax W, scale x, scale W
+        amax_x, amax_w, sx, sw = stats[0:1], stats[1:2], stats[2:3], stats[3:4]
+        fp8_quantize_many([(x2, T * K, FP8_E4M3, rings[0], x8, amax_x, sx),
+                           (w, N * K, FP8_E4M3, rings[1], w8, amax_w, sw)])
         y = torch.empty(T, N, dtype=torch.bfloat16, device=x.device)
         b = bias.contiguous() if bias is not None else None
         fp8_mm(x8, FP8_E4M3, w8, FP8_E4M3, sx, sw, FP8_NT, T, N, K, 1, 0, 0, 0, b, None, 0, y)
