@@ -43,7 +43,6 @@
 
 #include <algorithm>
 #include <mutex>
-#include <vector>
 
 #include "common.cuh"
 #include "sm100.cuh"
@@ -1213,25 +1212,36 @@ fp8_status launch_group(const GroupTab<true>& g, int total_units, cudaStream_t s
 // rounds of `grid`, alternating direction (unit_of), so the launch lasts as
 // long as its busiest CTA; this is that CTA's k-blocks (times the per-k-block
 // cost of the tile width) plus one exposed epilogue, the same cost model as a
-// single problem's choice.
+// single problem's choice. Past a few thousand units the rounds even out and
+// the estimate is rounds x the longest K.
 inline int choose_group_bn(const int64_t* M, const int64_t* N, const int64_t* kb, int count, int64_t sms) {
+    constexpr int64_t kMaxSlots = 1024, kSimUnits = 8192;
     int best_bn = 256;
     double best = 1e30;
     for (int bn : {256, 128}) {
         const double t_k = bn == 256 ? 0.48 : 0.40, t_epi = bn == 256 ? 2.0 : 1.0;
-        int64_t total = 0;
-        for (int i = 0; i < count; ++i) total += ((M[i] + BM - 1) / BM) * ((N[i] + bn - 1) / bn);
-        const int64_t grid = total < sms ? total : sms;
-        std::vector<int64_t> load(size_t(grid), 0);
-        int64_t u = 0;
+        int64_t total = 0, kb_max = 0;
         for (int i = 0; i < count; ++i) {
-            const int64_t tiles = ((M[i] + BM - 1) / BM) * ((N[i] + bn - 1) / bn);
-            for (int64_t k = 0; k < tiles; ++k, ++u) {
-                const int64_t round = u / grid, pos = u - round * grid;
-                load[size_t((round & 1) ? grid - 1 - pos : pos)] += kb[i];
-            }
+            total += ((M[i] + BM - 1) / BM) * ((N[i] + bn - 1) / bn);
+            kb_max = kb[i] > kb_max ? kb[i] : kb_max;
         }
-        const int64_t worst = *std::max_element(load.begin(), load.end());
+        const int64_t slots = sms < kMaxSlots ? sms : kMaxSlots;
+        const int64_t grid = total < slots ? total : slots;
+        int64_t worst = 0;
+        if (total > kSimUnits) {
+            worst = ((total + grid - 1) / grid) * kb_max;
+        } else {
+            int64_t load[kMaxSlots] = {0};
+            int64_t u = 0;
+            for (int i = 0; i < count; ++i) {
+                const int64_t tiles = ((M[i] + BM - 1) / BM) * ((N[i] + bn - 1) / bn);
+                for (int64_t k = 0; k < tiles; ++k, ++u) {
+                    const int64_t round = u / grid, pos = u - round * grid;
+                    load[(round & 1) ? grid - 1 - pos : pos] += kb[i];
+                }
+            }
+            for (int64_t c = 0; c < grid; ++c) worst = load[c] > worst ? load[c] : worst;
+        }
         const double c = double(worst) * t_k + t_epi;
         if (c < best) { best = c; best_bn = bn; }
     }
