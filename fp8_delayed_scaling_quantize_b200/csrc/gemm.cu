@@ -89,15 +89,20 @@ struct GemmParams {
 };
 
 // Grouped launch (fp8_mm_grouped): several independent problems share one
-// persistent grid. Work units [unit_end of the previous problem, unit_end)
-// are the tiles of problem i; each role looks its unit's problem up here.
+// persistent grid. Work units [unit_end of the previous entry, unit_end) are
+// the tiles of entry i; each role looks its unit's entry up here. An entry is
+// a problem, or a column range of one: the host may give a problem's last
+// columns their own entry with 128-wide tiles, so that the tiles of the
+// grid's last round are cheaper.
 constexpr int kMaxGroup = FP8_MM_MAX_GROUP;
+constexpr int kMaxEntries = kMaxGroup + 1;
 struct GroupProblem {
     CUtensorMap ta, tb, tc;  // operand maps and the output's store map
     int M, N, k_blocks, m_tiles, n_tiles, unit_end;
     int a_mn, b_mn;
     uint32_t idesc;
     int bias_kind, bias_fmt, tma_store, vec_store;
+    int bn, n_base;  // this entry's tile width (128 or the launch's BN) and first output column
     const float* sa;
     const float* sb;
     const void* bias;
@@ -108,7 +113,7 @@ template <bool GROUP>
 struct GroupTab {};  // single-problem launches carry no table
 template <>
 struct GroupTab<true> {
-    GroupProblem q[kMaxGroup];
+    GroupProblem q[kMaxEntries];
     int count;
 };
 
@@ -382,6 +387,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                 bool a_mn = A_MN, b_mn = B_MN;
                 TileWalk w = walk;
                 int kbs = k_blocks;
+                int ebn = BN, n_base = 0;  // the unit's tile width and first column
                 if constexpr (GROUP) {
                     const GroupProblem& q = group_problem(grp, u, t);
                     map_a = &q.ta;
@@ -390,6 +396,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                     b_mn = q.b_mn;
                     w = {q.m_tiles, q.n_tiles, walk.group_m};
                     kbs = q.k_blocks;
+                    ebn = q.bn;
+                    n_base = q.n_base;
                 }
                 const int kb0 = GROUP ? 0 : (u - t * split) * kb_per;
                 const int kb1 = GROUP ? kbs : min(k_blocks, kb0 + kb_per);
@@ -398,11 +406,12 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                 const int ba = a_bcast ? 0 : b;
                 const int bb = b_bcast ? 0 : b;
                 const int m0 = mb * BM * CTAS + int(rank) * BM;
-                const int n0 = nb * BN + int(rank) * (BN / CTAS);
+                const int n0 = n_base + nb * ebn + int(rank) * (BN / CTAS);
+                const uint32_t stage_tx = GROUP ? uint32_t(L::kABytes + ebn * BK) : uint32_t(L::kStageTx);
                 for (int kb = kb0; kb < kb1; ++kb) {
                     if (!wait_bounded(bar_empty + 8 * stage, phase ^ 1)) { ok = false; break; }
                     const uint32_t full = bar_full + 8 * stage;
-                    if (leader) mbar_arrive_expect_tx(full, L::kStageTx);
+                    if (leader) mbar_arrive_expect_tx(full, stage_tx);
                     const uint32_t da = s_a + stage * L::kABytes;
                     const uint32_t db = s_b + stage * L::kBBytes;
                     if (CTAS == 1) {
@@ -411,7 +420,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                         if (b_mn) {
 #pragma unroll
                             for (int h = 0; h < BN / 128; ++h)
-                                tma_load_3d(db + h * 128 * BK, map_b, full, n0 + h * 128, kb * BK, bb);
+                                if (h * 128 < ebn) tma_load_3d(db + h * 128 * BK, map_b, full, n0 + h * 128, kb * BK, bb);
                         } else {
                             tma_load_3d(db, map_b, full, kb * BK, n0, bb);
                         }
@@ -511,9 +520,12 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             int t = u / split;
             const int split_id = u - t * split;
             TileWalk w = walk;
+            int ebn = BN, n_base = 0;  // the unit's tile width and first column
             if constexpr (GROUP) {
                 const GroupProblem& q = group_problem(grp, u, t);
                 w = {q.m_tiles, q.n_tiles, walk.group_m};
+                ebn = q.bn;
+                n_base = q.n_base;
                 M = q.M;
                 N = q.N;
                 tma_store = q.tma_store;
@@ -534,8 +546,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             if (HAS_BIAS && !SWAP) {
                 // the tile's BN bias values, dequantized once into shared memory
                 epilogue_bar();  // the previous tile's readers are done
-                for (int j = etid; j < BN; j += kEpiThreads) {
-                    const int col = nb * BN + j;
+                for (int j = etid; j < ebn; j += kEpiThreads) {
+                    const int col = n_base + nb * ebn + j;
                     float v = 0.0f;
                     if (col < N && bias_kind != 0) {  // a grouped launch may mix problems with and without bias
                         if (bias_kind == 1) {
@@ -614,8 +626,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             uint16_t* orow = SWAP ? out_base + int64_t(b) * p.stride_c + row
                                   : out_base + int64_t(b) * p.stride_c + int64_t(row) * N;
 #pragma unroll 1
-            for (int c = 0; c < BN / CW; ++c) {
-                const int col0 = nb * BN + c * CW;
+            for (int c = 0; c < ebn / CW; ++c) {
+                const int col0 = n_base + nb * ebn + c * CW;
                 if (col0 >= N) break;  // uniform over the epilogue warps
                 uint32_t r[CW];
                 tmem_ld<CW>(t_row + c * CW, r);
@@ -1080,6 +1092,10 @@ namespace fp8lite {
 namespace {
 
 // The FP8 output of fp8_mm_out8 (none for the bf16 entry points).
+inline int choose_group_bn(const int64_t* M, const int64_t* N, const int64_t* kb, int count, int64_t sms);
+inline int choose_narrow_tail(const int64_t* M, const int64_t* N, const int64_t* kb, int count, int64_t sms);
+fp8_status mm_grouped_impl(const fp8_mm_problem* probs, int32_t count, void* stream);
+
 struct Out8 {
     bool on;
     fp8_fmt fmt;
@@ -1151,6 +1167,19 @@ fp8_status mm_impl(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8, fp8_fmt fb,
         p.tma_store = p.vec_store;
     }
     cudaStream_t st = as_stream(stream);
+    // One problem whose 128 x 256 tiles leave the persistent grid's last round
+    // part-empty runs as a grouped launch of one, where its rightmost columns
+    // can take 128-wide tiles (choose_narrow_tail); the result is the same.
+    if (!o8.on && batch == 1 && split_k <= 1 && !swap_ab(M, N, layout)) {
+        const TileChoice tc = choose_tile(M, N, K, 1, b_mn, sm_count(), split_k);
+        const int64_t kb1 = (K + BK - 1) / BK;
+        if (!tc.pair && tc.bn == 256 && tc.split == 1 && choose_group_bn(&M, &N, &kb1, 1, sm_count()) == 256 &&
+            choose_narrow_tail(&M, &N, &kb1, 1, sm_count()) > 0) {
+            const fp8_mm_problem one = {a8, b8, sa, sb, bias, bias_scale, out, M, N, K,
+                                        int32_t(fa), int32_t(fb), int32_t(layout), int32_t(bias_fmt)};
+            return mm_grouped_impl(&one, 1, stream);
+        }
+    }
     if (!o8.on && swap_ab(M, N, layout))
         return layout == FP8_NN ? dispatch_swap<true>(a8, fa, b8, fb, M, N, K, batch, stride_a, stride_b, p, workspace,
                                                       workspace_bytes, split_k, st)
@@ -1248,6 +1277,51 @@ inline int choose_group_bn(const int64_t* M, const int64_t* N, const int64_t* kb
     return best_bn;
 }
 
+// How many of the last problem's 256-wide column tiles (counted from its
+// right edge) to run as 128-wide tiles in a 256-wide grouped launch. The
+// launch's last round often holds fewer tiles than there are CTAs; a 128-wide
+// tile costs about 0.28 us per k-block against 0.45 us for a 256-wide one
+// (measured on B200 with this kernel), so narrower tiles at the end shorten
+// the busiest CTA. Each choice is evaluated on the exact unit-to-CTA
+// assignment (unit_of); 0 keeps every tile 256 wide.
+inline int choose_narrow_tail(const int64_t* M, const int64_t* N, const int64_t* kb, int count, int64_t sms) {
+    constexpr int64_t kMaxSlots = 1024, kSimUnits = 8192;
+    const int last = count - 1;
+    const int64_t n256 = (N[last] + 255) / 256;
+    int best_k = 0;
+    double best = 1e30;
+    for (int64_t k = 0; k <= n256; ++k) {
+        const int64_t n1 = (n256 - k) * 256;  // columns left 256 wide
+        int64_t units[kMaxEntries], cost[kMaxEntries];  // per entry: tiles, and their cost in 0.01 us
+        int e = 0;
+        for (int i = 0; i < last; ++i, ++e) {
+            units[e] = ((M[i] + BM - 1) / BM) * ((N[i] + 255) / 256);
+            cost[e] = kb[i] * 45;
+        }
+        const int64_t mt = (M[last] + BM - 1) / BM;
+        units[e] = mt * (n1 / 256);
+        cost[e++] = kb[last] * 45;
+        units[e] = mt * ((N[last] - n1 + 127) / 128);
+        cost[e++] = kb[last] * 28;
+        int64_t total = 0;
+        for (int i = 0; i < e; ++i) total += units[i];
+        if (total > kSimUnits) return 0;
+        const int64_t slots = sms < kMaxSlots ? sms : kMaxSlots;
+        const int64_t grid = total < slots ? total : slots;
+        int64_t load[kMaxSlots] = {0};
+        int64_t u = 0;
+        for (int i = 0; i < e; ++i)
+            for (int64_t t = 0; t < units[i]; ++t, ++u) {
+                const int64_t round = u / grid, pos = u - round * grid;
+                load[(round & 1) ? grid - 1 - pos : pos] += cost[i];
+            }
+        int64_t worst = 0;
+        for (int64_t c = 0; c < grid; ++c) worst = load[c] > worst ? load[c] : worst;
+        if (double(worst) < best - 1e-9) { best = double(worst); best_k = int(k); }
+    }
+    return best_k;
+}
+
 fp8_status mm_grouped_impl(const fp8_mm_problem* probs, int32_t count, void* stream) {
     if (!probs || count < 1 || count > kMaxGroup) return FP8_ERR_INVALID_ARG;
     for (int i = 0; i < count; ++i) {
@@ -1278,42 +1352,55 @@ fp8_status mm_grouped_impl(const fp8_mm_problem* probs, int32_t count, void* str
         kb[i] = (probs[order[i]].K + BK - 1) / BK;
     }
     const int bn = choose_group_bn(M, N, kb, count, sm_count());
+    // entries: every problem with bn-wide tiles; in a 256-wide launch the last
+    // problem's rightmost columns may form one more entry with 128-wide tiles
+    const int narrow = bn == 256 ? choose_narrow_tail(M, N, kb, count, sm_count()) : 0;
     GroupTab<true> g = {};
-    g.count = count;
     int64_t units = 0;
     bool any_bias = false;
+    int e = 0;
     for (int i = 0; i < count; ++i) {
         const fp8_mm_problem& q = probs[order[i]];
-        GroupProblem& d = g.q[i];
         const bool a_mn = q.layout == FP8_TN, b_mn = q.layout != FP8_NT;
-        const bool ok = (a_mn ? make_map(&d.ta, q.a8, q.M, q.K, 1, 0, 128, BK)
-                              : make_map(&d.ta, q.a8, q.K, q.M, 1, 0, BK, BM)) &&
-                        (b_mn ? make_map(&d.tb, q.b8, q.N, q.K, 1, 0, 128, BK)
-                              : make_map(&d.tb, q.b8, q.K, q.N, 1, 0, BK, uint32_t(bn)));
-        if (!ok) return FP8_ERR_CUDA;
-        d.M = int(q.M);
-        d.N = int(q.N);
-        d.k_blocks = int(kb[i]);
-        d.m_tiles = int((q.M + BM - 1) / BM);
-        d.n_tiles = int((q.N + bn - 1) / bn);
-        units += int64_t(d.m_tiles) * d.n_tiles;
-        if (units >= (int64_t(1) << 31)) return FP8_ERR_UNSUPPORTED;
-        d.unit_end = int(units);
-        d.a_mn = a_mn;
-        d.b_mn = b_mn;
-        d.idesc = sm100::instr_desc_f8(q.fmt_a, q.fmt_b, a_mn, b_mn, BM, bn);
-        d.bias_kind = q.bias ? (q.bias_scale ? 2 : 1) : 0;
-        d.bias_fmt = q.bias_fmt;
-        any_bias = any_bias || q.bias;
-        d.vec_store = (q.N % 8 == 0) && aligned(q.out, 16);
-        d.tma_store = d.vec_store;
-        if (d.tma_store && !make_out_map(&d.tc, q.out, q.N, q.M, 1, 0)) return FP8_ERR_CUDA;
-        d.sa = q.sa;
-        d.sb = q.sb;
-        d.bias = q.bias;
-        d.bias_scale = q.bias_scale;
-        d.out = static_cast<uint16_t*>(q.out);
+        // column ranges of this problem: [0, n1) at bn, [n1, N) at 128
+        const int64_t n1 = (i == count - 1 && narrow > 0) ? ((q.N + 255) / 256 - narrow) * 256 : q.N;
+        for (int part = 0; part < 2; ++part) {
+            const int64_t c0 = part == 0 ? 0 : n1, c1 = part == 0 ? n1 : q.N;
+            if (c1 <= c0) continue;
+            const int ebn = part == 0 ? bn : 128;
+            GroupProblem& d = g.q[e++];
+            const bool ok = (a_mn ? make_map(&d.ta, q.a8, q.M, q.K, 1, 0, 128, BK)
+                                  : make_map(&d.ta, q.a8, q.K, q.M, 1, 0, BK, BM)) &&
+                            (b_mn ? make_map(&d.tb, q.b8, q.N, q.K, 1, 0, 128, BK)
+                                  : make_map(&d.tb, q.b8, q.K, q.N, 1, 0, BK, uint32_t(ebn)));
+            if (!ok) return FP8_ERR_CUDA;
+            d.M = int(q.M);
+            d.N = int(q.N);
+            d.k_blocks = int(kb[i]);
+            d.m_tiles = int((q.M + BM - 1) / BM);
+            d.n_tiles = int((c1 - c0 + ebn - 1) / ebn);
+            d.bn = ebn;
+            d.n_base = int(c0);
+            units += int64_t(d.m_tiles) * d.n_tiles;
+            if (units >= (int64_t(1) << 31)) return FP8_ERR_UNSUPPORTED;
+            d.unit_end = int(units);
+            d.a_mn = a_mn;
+            d.b_mn = b_mn;
+            d.idesc = sm100::instr_desc_f8(q.fmt_a, q.fmt_b, a_mn, b_mn, BM, ebn);
+            d.bias_kind = q.bias ? (q.bias_scale ? 2 : 1) : 0;
+            d.bias_fmt = q.bias_fmt;
+            any_bias = any_bias || q.bias;
+            d.vec_store = (q.N % 8 == 0) && aligned(q.out, 16);
+            d.tma_store = d.vec_store;
+            if (d.tma_store && !make_out_map(&d.tc, q.out, q.N, q.M, 1, 0)) return FP8_ERR_CUDA;
+            d.sa = q.sa;
+            d.sb = q.sb;
+            d.bias = q.bias;
+            d.bias_scale = q.bias_scale;
+            d.out = static_cast<uint16_t*>(q.out);
+        }
     }
+    g.count = e;
     cudaStream_t st = as_stream(stream);
     if (bn == 256)
         return any_bias ? launch_group<256, 4, true>(g, int(units), st) : launch_group<256, 4, false>(g, int(units), st);

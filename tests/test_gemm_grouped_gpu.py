@@ -125,6 +125,31 @@ def test_grouped_three_layouts_ragged_mid_size(g):
         p.check_same_as_fp8_mm(g, f"mid-size problem {i} vs fp8_mm")
 
 
+def test_grouped_narrow_tail_ragged(g):
+    """Two problems whose 128 x 256 tiles leave the grid's last round short:
+    the launch runs the last problem's rightmost columns as 128-wide tiles
+    (a second entry whose N edge is ragged). Full comparison with the oracle,
+    with a bias on the split problem."""
+    specs = [(NT, 2048, 1936, 384, E4M3, E4M3, 1), (NT, 1024, 1000, 640, E4M3, E5M2, 0)]
+    probs = [Prob(*s[:6], seed=1700 + 10 * i, bias_kind=s[6]) for i, s in enumerate(specs)]
+    _run(probs)
+    for i, p in enumerate(probs):
+        p.check_full(g, f"narrow tail problem {i}")
+        p.check_same_as_fp8_mm(g, f"narrow tail problem {i} vs fp8_mm")
+
+
+def test_fp8_mm_routed_through_narrow_tail(g):
+    """fp8_mm of a shape whose last round of 128 x 256 tiles is short (QKV
+    forward of the linear stack, and a ragged variant) runs as a grouped launch
+    with a 128-wide tail; the output is compared in full with the oracle."""
+    for spec in ((NT, 2048, 3072, 1024, E4M3, E4M3, 0), (NT, 1000, 3100, 512, E4M3, E4M3, 2)):
+        p = Prob(*spec[:6], seed=1800, bias_kind=spec[6])
+        out = p.single(g)
+        torch.cuda.synchronize()
+        p.out[:p.M * p.N].copy_(out[:p.M * p.N])
+        p.check_full(g, f"routed fp8_mm {spec[:4]}")
+
+
 def _sample_idx(M, N, seed):
     rng = np.random.default_rng(seed)
     i = rng.integers(0, M, 2048)
