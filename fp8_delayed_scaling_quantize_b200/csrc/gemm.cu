@@ -466,24 +466,23 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                 if (!wait_bounded(bar_tempty + 8 * buf, acc_phase ^ 1)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + buf * BN;
+                const uint64_t a_desc0 = a_mn ? smem_desc_sw128(s_a, 128 * BK, 1024) : smem_desc_sw128(s_a, 16, 1024);
+                const uint64_t b_desc0 = b_mn ? smem_desc_sw128(s_b, 128 * BK, 1024) : smem_desc_sw128(s_b, 16, 1024);
                 for (int kb = kb0; kb < kb1; ++kb) {
                     // the stage's operands arrive through the async proxy and
                     // complete on this barrier: the MMAs may read them without
                     // a tcgen05 fence (that is needed only after the epilogue's
                     // hand-back of the accumulator, above)
                     if (!wait_bounded(bar_full + 8 * stage, phase)) { ok = false; break; }
-                    const uint32_t da = s_a + stage * L::kABytes;
-                    const uint32_t db = s_b + stage * L::kBBytes;
-#pragma unroll
-                    for (int j = 0; j < BK / 32; ++j) {
-                        // K-major: the 32-byte K step moves inside the swizzle atom;
-                        // MN-major: it skips 32 rows of 128 bytes (4 atoms).
-                        const uint64_t adesc = a_mn ? smem_desc_sw128(da + j * 32 * 128, 128 * BK, 1024)
-                                                    : smem_desc_sw128(da + j * 32, 16, 1024);
-                        const uint64_t bdesc = b_mn ? smem_desc_sw128(db + j * 32 * 128, 128 * BK, 1024)
-                                                    : smem_desc_sw128(db + j * 32, 16, 1024);
-                        mma_f8f6f4<CTAS>(d_tmem, adesc, bdesc, id, kb != kb0 || j != 0);
-                    }
+                    // the stage's descriptors: stage 0's plus the stage offset in
+                    // the start-address field (16-byte units; no carry out of it,
+                    // shared memory is below 256 KB). Each next 32-deep K slice is
+                    // +32 bytes inside the swizzle atom (K-major) or 32 rows of
+                    // 128 bytes further (MN-major).
+                    const uint64_t adesc = a_desc0 + uint64_t(stage) * (L::kABytes >> 4);
+                    const uint64_t bdesc = b_desc0 + uint64_t(stage) * (L::kBBytes >> 4);
+                    mma_kblock_f8f6f4<CTAS>(d_tmem, adesc, bdesc, a_mn ? 256u : 2u, b_mn ? 256u : 2u, id,
+                                            kb != kb0);
                     // release the stage (in both CTAs of a pair)
                     if (CTAS == 1) mma_commit(bar_empty + 8 * stage);
                     else           mma_commit_pair(bar_empty + 8 * stage);

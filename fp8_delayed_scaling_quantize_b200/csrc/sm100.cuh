@@ -165,22 +165,41 @@ __device__ __forceinline__ void tc_fence_after() {
 // D[tmem] (+)= A[smem desc] * B[smem desc], FP8 operands, fp32 accumulate.
 // CG = 2: issued by the pair's leader; each CTA supplies its half of A (its
 // 128 rows) and of B (N/2 columns) and holds its rows of D.
+//
+// The four MMAs of one 128-deep k-block (K = 32 each), issued from one asm
+// block: descriptors of the first K slice in adesc / bdesc, each next slice
+// at +a_step / +b_step in the descriptors' start-address field (16-byte
+// units). The first MMA accumulates only if `accumulate`, the others always.
 template <int CG>
-__device__ __forceinline__ void mma_f8f6f4(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                           uint32_t accumulate) {
+__device__ __forceinline__ void mma_kblock_f8f6f4(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint64_t a_step,
+                                                  uint64_t b_step, uint32_t idesc, uint32_t accumulate) {
     if (CG == 1)
         asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "setp.ne.b32 p, %4, 0;\n\t"
-            "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+            "{\n\t.reg .pred p, q;\n\t.reg .b64 a, b;\n\t"
+            "setp.ne.b32 p, %6, 0;\n\t"
+            "setp.eq.b32 q, %6, %6;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %5, p;\n\t"
+            "add.s64 a, %1, %3;\n\tadd.s64 b, %2, %4;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %5, q;\n\t"
+            "add.s64 a, a, %3;\n\tadd.s64 b, b, %4;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %5, q;\n\t"
+            "add.s64 a, a, %3;\n\tadd.s64 b, b, %4;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %5, q;\n\t}" ::"r"(tmem_d),
+            "l"(adesc), "l"(bdesc), "l"(a_step), "l"(b_step), "r"(idesc), "r"(accumulate)
             : "memory");
     else
         asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "setp.ne.b32 p, %4, 0;\n\t"
-            "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+            "{\n\t.reg .pred p, q;\n\t.reg .b64 a, b;\n\t"
+            "setp.ne.b32 p, %6, 0;\n\t"
+            "setp.eq.b32 q, %6, %6;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %5, p;\n\t"
+            "add.s64 a, %1, %3;\n\tadd.s64 b, %2, %4;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], a, b, %5, q;\n\t"
+            "add.s64 a, a, %3;\n\tadd.s64 b, b, %4;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], a, b, %5, q;\n\t"
+            "add.s64 a, a, %3;\n\tadd.s64 b, b, %4;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], a, b, %5, q;\n\t}" ::"r"(tmem_d),
+            "l"(adesc), "l"(bdesc), "l"(a_step), "l"(b_step), "r"(idesc), "r"(accumulate)
             : "memory");
 }
 
