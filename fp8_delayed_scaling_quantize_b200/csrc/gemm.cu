@@ -221,12 +221,14 @@ struct Smem {
     static constexpr int kBBytes = (BN / CTAS) * BK;
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kStageTx = CTAS * kStageBytes;  // bytes landing on the leader's full barrier
-    // two 128-row x 32-column bf16 staging tiles (64-byte swizzle), used in
-    // turn; 16 KB in all, so that a waiting kernel's small blocks still fit
-    // on the SM beside this CTA
+    // three 128-row x 32-column bf16 staging tiles (64-byte swizzle), used in
+    // turn, so that a chunk waits only for the store two chunks back; 24 KB
+    // in all, so that a waiting kernel's small blocks still fit on the SM
+    // beside this CTA
+    static constexpr int kStgBufs = 3;
     static constexpr int kStgBytes = BM * 32 * 2;
     static constexpr int kStgOffset = STAGES * kStageBytes;  // a multiple of 1024
-    static constexpr int kBiasOffset = kStgOffset + 2 * kStgBytes;  // BN fp32 bias values
+    static constexpr int kBiasOffset = kStgOffset + kStgBufs * kStgBytes;  // BN fp32 bias values
     static constexpr int kBarOffset = kBiasOffset + BN * 4;
     // full[S], empty[S], tmem_full[2], tmem_empty[2], then the TMEM slot and the split ticket
     static constexpr int kBytes = kBarOffset + (2 * STAGES + 4) * 8 + 16;
@@ -499,7 +501,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         const int etid = threadIdx.x - 64;  // 0 .. kEpiThreads-1
         const bool store_lead = etid == 0;  // issues the TMA stores
         const uint32_t stg0 = s_base + L::kStgOffset;
-        int n_st = 0;  // TMA stores issued so far (they alternate between the two staging tiles)
+        int n_st = 0;  // TMA stores issued so far (they take the staging tiles in turn)
         float inv = (1.0f / __ldg(p.sa)) * (1.0f / __ldg(p.sb));
         int bias_kind = p.bias_kind, bias_fmt = p.bias_fmt;
         const void* bias_ptr = p.bias;
@@ -708,7 +710,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                         // piece j of row r at (j ^ (r / 2 mod 4)) * 16, so the 8
                         // lanes of a store phase hit distinct banks); then one TMA
                         // store, which clips the M / N tails of the output
-                        const uint32_t stg = stg0 + (n_st & 1) * L::kStgBytes;
+                        const uint32_t stg = stg0 + uint32_t(n_st % L::kStgBufs) * L::kStgBytes;
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
                             const uint32_t addr = stg + row_in_tile * 64 + ((j ^ ((row_in_tile >> 1) & 3)) << 4);
@@ -720,9 +722,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                                          : "memory");
                         }
                         fence_proxy_async_smem();
-                        // the previous store has read the other tile, which the next
-                        // block reuses; the barrier publishes that and this block
-                        if (store_lead) bulk_wait_read<0>();
+                        // the store two blocks back has read its tile, which the next
+                        // block reuses (only the newest store may still be reading);
+                        // the barrier publishes that and this block
+                        if (store_lead) bulk_wait_read<L::kStgBufs - 2>();
                         epilogue_bar();
                         if (store_lead) {
                             tma_store_3d(map_c, stg, col0, m0, b);
