@@ -297,9 +297,10 @@ __device__ __forceinline__ bool epilogue_bar_or(bool v) {
 // become a 128 x 32 bf16 tile in shared memory that one thread writes with a
 // single TMA store (8 stores for a 128 x 256 tile).
 //
-// GROUP: the units are the tiles of up to kMaxGroup problems (one SM per
-// tile, no split, no batches); operand majors, maps, scales, bias and output
-// come from the group table per unit, A_MN / B_MN only give the defaults.
+// GROUP: the units are the tiles of up to kMaxEntries table entries (one SM
+// per tile, no split, no batches); operand majors, maps, tile width, first
+// column, scales, bias and output come from the entry of each unit, A_MN /
+// B_MN only give the defaults and BN is the widest tile.
 template <int BN, bool A_MN, bool B_MN, int STAGES, bool HAS_BIAS, int CTAS, bool SPLIT, bool SWAP, bool OUT8,
           bool GROUP = false>
 __global__ void __maxnreg__(168)
