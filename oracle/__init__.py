@@ -33,7 +33,9 @@ Parity pins: every function here is pinned in ``tests/test_oracle_*.py``
 against facts that do not come from this code (OFP8 boundary values, an
 independent library cast, exact rational brute force, hand-computed ring
 tables). One reading is **parity unpinned**: the treatment of NaN inputs in
-the amax (NaN is ignored); no configuration contains NaN.
+the amax (NaN is ignored), which the pages do not fix; no configuration
+contains NaN. The GPU tests hold the kernel to this reading on every bf16
+pattern, NaNs included.
 """
 
 from .codec import (  # noqa: F401

@@ -33,8 +33,10 @@ Readings taken where the pages are silent:
 * the ring holds H = 16 entries, starts at hist = 0, idx = 0, scale = 1.
 * a window maximum that is 0 or non-finite keeps the previous scale.
 * the window includes the amax just written.
-* NaN inputs are ignored by the amax (**parity unpinned**: no configuration
-  contains NaN).
+* NaN inputs are ignored by the amax (**parity unpinned** for this one
+  reading: the pages fix no NaN behaviour and no configuration contains NaN;
+  the amax itself is pinned on finite inputs, and the GPU kernel is compared
+  with this reading on every bf16 pattern, NaNs included).
 """
 
 import numpy as np
