@@ -46,7 +46,12 @@ def _run_case(g, layout, M, N, K, fa, fb, out_fmt, seed, batch=1, bcast_b=False,
     stride_b = 0 if bcast_b else N * K
     ad, bd = a8.cuda(), b8.cuda()
     ring = g.new_ring(1.0)
+    # ref folds the GPU's amax: the fp32 y that the amax is taken over is not
+    # bit-defined (only held to the GEMM tolerance), so the ring's fold is
+    # checked bit for bit given that amax; ref_own folds the oracle's own
+    # amax and bounds the published scale by the amax tolerance
     ref = oracle.DelayedRing(1.0)
+    ref_own = oracle.DelayedRing(1.0)
     for step, sa in enumerate((4.0, 0.5, 16.0)):
         sb = 1.5
         s_used = np.float32(ref.scale)
@@ -68,10 +73,16 @@ def _run_case(g, layout, M, N, K, fa, fb, out_fmt, seed, batch=1, bcast_b=False,
         assert not bad.any(), f"step {step}: {int(bad.sum())} codes outside the bound"
         assert (codes == q).mean() > 0.98, step  # all but boundary cases give the oracle's code itself
         a_gpu = g.f32(amax)[0]
-        assert abs(float(a_gpu) - float(amax_want)) <= 2.0 ** -16 * float(s_abs.max()) + 2.0 ** -22 * float(amax_want)
+        a_tol = 2.0 ** -16 * float(s_abs.max()) + 2.0 ** -22 * float(amax_want)
+        assert abs(float(a_gpu) - float(amax_want)) <= a_tol
         ref.fold(a_gpu, out_fmt)
+        ref_own.fold(amax_want, out_fmt)
         hist, rs, idx, acc, ticket = g.ring_state(ring)
         assert np.array_equal(hist, ref.hist) and rs == ref.scale and idx == ref.idx, step
+        # the window maxima differ by at most a_tol, so the published scales
+        # differ by that relative amount plus one fp32 rounding
+        rel = a_tol / float(np.max(ref_own.hist))
+        assert abs(float(rs) / float(ref_own.scale) - 1.0) <= rel / (1.0 - rel) + 2.0 ** -23, step
         assert acc == 0 and ticket == 0
         for b in range(batch):
             assert (got[b * stride_c + M * N: (b + 1) * stride_c] == 0xEE).all()
