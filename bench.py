@@ -177,14 +177,21 @@ class ClockSampler:
 class Stack:
     """Device buffers and the C-ABI calls of one step of the linear stack."""
 
-    def __init__(self, fp8, n_sets=N_SETS, dev="cuda"):
+    def __init__(self, fp8, n_sets=N_SETS, dev="cuda", tokens=W.TOKENS):
+        """tokens: a multiple of the workload's 2048; above it, each set's x
+        and g are the workload's draws repeated along the token dimension (the
+        values do not change the timing)."""
         self.fp8 = fp8
         self.dev = dev
+        self.tokens = tokens
+        rep = tokens // W.TOKENS
+        assert rep * W.TOKENS == tokens
         self.sets = []
         for s in range(n_sets):
             ts = W.stack_tensors(s)
-            self.sets.append([{k: v.to(dev) for k, v in t.items()} for t in ts])
-        T = W.TOKENS
+            self.sets.append([{k: (v.to(dev).repeat(rep, 1) if k != "w" and rep > 1 else v.to(dev))
+                               for k, v in t.items()} for t in ts])
+        T = tokens
         self.lin = []
         # all 12 rings in one [12, 20] tensor, so the data-parallel exchange
         # all-reduces their amax words in one message and folds them in one launch
@@ -204,8 +211,8 @@ class Stack:
             L["dx"] = torch.empty(T * d_in, dtype=torch.bfloat16, device=dev)
             L["dw"] = torch.empty(d_out * d_in, dtype=torch.bfloat16, device=dev)
             self.lin.append(L)
-        self.flops = W.stack_flops()
-        self.q_elems = W.stack_quant_elems()
+        self.flops = sum(3 * 2 * T * di * do for _, di, do in W.LINEARS)
+        self.q_elems = sum(T * di + do * di + T * do for _, di, do in W.LINEARS)
         self.split_k = 0
         self.ws = [None, None]
         self.group_bwd = True
@@ -260,7 +267,7 @@ class Stack:
 
     def gemm_calls(self, li):
         L = self.lin[li]
-        T, di, do = W.TOKENS, L["d_in"], L["d_out"]
+        T, di, do = self.tokens, L["d_in"], L["d_out"]
         q, sc = L["q"], L["scale"]
         return [
             # forward y = x W^T: NT, M=T, N=d_out, K=d_in
@@ -273,7 +280,7 @@ class Stack:
 
     def gemm_flops(self, li):
         L = self.lin[li]
-        return 2 * W.TOKENS * L["d_in"] * L["d_out"]
+        return 2 * self.tokens * L["d_in"] * L["d_out"]
 
     def grouped_call(self, s):
         """The step-start quantize of every linear's W and of the first x,
@@ -350,6 +357,78 @@ def gemm_algorithmic_bytes(layout, M, N, K):
     return M * K + N * K + 2 * M * N
 
 
+def breakdown(fp8, stack, stream, reps, rotate):
+    """Per-launch device time of each of the step's kernels, back to back.
+
+    rotate=False repeats each call on the step's own buffers (L2-resident);
+    rotate=True gives call i copies number i mod k of every input and output,
+    k sized so that the copies exceed twice the L2, so each launch reads its
+    inputs from HBM as it does inside the step."""
+    dev = stack.dev
+    q_ms = g_ms = 0.0
+    q_elems = g_flops = g_bytes = 0
+    n_g = n_q = 0
+    per_shape, per_tensor = {}, {}
+    names = ("x", "w", "g")
+    for li in range(len(stack.lin)):
+        L = stack.lin[li]
+        calls = [("quantize", c, names[i]) for i, c in enumerate(stack.quant_calls(0, li))]
+        if stack.use_group_bwd():
+            calls += [("gemm", stack.gemm_calls(li)[0], None), ("pair", stack.bwd_pair(li), None)]
+        else:
+            calls += [("gemm", c, None) for c in stack.gemm_calls(li)]
+        for kind, c, role in calls:
+            if kind == "quantize":
+                x, n, fmt, ring, q, am, sc = c
+                k = _slots(3 * n) if rotate else 1
+                X = [x] + [x.clone() for _ in range(k - 1)]
+                Q = [q] + [torch.empty_like(q) for _ in range(k - 1)]
+                call = lambda i: fp8.fp8_quantize(X[i % k], n, fmt, ring, Q[i % k], am, sc, stream=stream)
+            elif kind == "pair":
+                dx, dw = c
+                g8, w8, x8 = dx[0], dx[2], dw[2]
+                nbytes = g8.numel() + w8.numel() + x8.numel() + 2 * (dx[13].numel() + dw[13].numel())
+                k = _slots(nbytes) if rotate else 1
+                G = [g8] + [g8.clone() for _ in range(k - 1)]
+                Wc = [w8] + [w8.clone() for _ in range(k - 1)]
+                Xc = [x8] + [x8.clone() for _ in range(k - 1)]
+                DX = [dx[13]] + [torch.empty_like(dx[13]) for _ in range(k - 1)]
+                DW = [dw[13]] + [torch.empty_like(dw[13]) for _ in range(k - 1)]
+                call = lambda i: fp8.fp8_mm_grouped(
+                    [(G[i % k],) + dx[1:2] + (Wc[i % k],) + dx[3:13] + (DX[i % k],),
+                     (G[i % k],) + dw[1:2] + (Xc[i % k],) + dw[3:13] + (DW[i % k],)], stream=stream)
+            else:
+                M, N, K = c[7:10]
+                k = _slots(gemm_algorithmic_bytes(c[6], M, N, K)) if rotate else 1
+                A = [c[0]] + [c[0].clone() for _ in range(k - 1)]
+                B = [c[2]] + [c[2].clone() for _ in range(k - 1)]
+                C = [c[17]] + [torch.empty_like(c[17]) for _ in range(k - 1)]
+                call = lambda i: stack.mm((A[i % k],) + c[1:2] + (B[i % k],) + c[3:17] + (C[i % k],), stream)
+            ms = _time_us(stream, call, reps) * 1e-3
+            if kind == "quantize":
+                q_ms += ms
+                q_elems += c[1]
+                n_q += 1
+                per_tensor[f"{L['name']}.{role} {c[1]}"] = (ms, c[1])
+            elif kind == "pair":
+                g_ms += ms
+                f = sum(2 * M * N * K for (M, N, K) in (q[7:10] for q in c))
+                g_flops += f
+                g_bytes += sum(gemm_algorithmic_bytes(q[6], *q[7:10]) for q in c)
+                n_g += 1
+                per_shape[" + ".join(f"{'NT NN TN'.split()[q[6]]} {q[7]}x{q[8]}x{q[9]}" for q in c)] = (ms, f)
+            else:
+                M, N, K = c[7:10]
+                g_ms += ms
+                g_flops += 2 * M * N * K
+                g_bytes += gemm_algorithmic_bytes(c[6], M, N, K)
+                n_g += 1
+                per_shape[f"{'NT NN TN'.split()[c[6]]} {M}x{N}x{K}"] = (ms, 2 * M * N * K)
+    torch.cuda.synchronize()
+    return {"q_ms": q_ms, "q_elems": q_elems, "n_q": n_q, "g_ms": g_ms, "g_flops": g_flops, "g_bytes": g_bytes,
+            "n_g": n_g, "per_shape": per_shape, "per_tensor": per_tensor}
+
+
 # ------------------------------------------------------------ our arm -------
 
 def run_ours(args, world, rank, local):
@@ -411,53 +490,18 @@ def run_ours(args, world, rank, local):
     # linear, and a grouped dX + dW launch per linear, or the two apart) is
     # repeated back to back between one event pair (the stream held while the
     # host enqueues), so the average is the kernel's steady-state cost on the
-    # stream, as inside the graph.
-    q_ms = g_ms = 0.0
-    q_elems = g_flops = g_bytes = 0
-    n_g = n_q = 0
-    per_shape = {}
-    reps = args.breakdown_reps
-    for li in range(len(stack.lin)):
-        calls = [("quantize", c) for c in stack.quant_calls(0, li)]
-        if stack.use_group_bwd():
-            calls += [("gemm", stack.gemm_calls(li)[0]), ("pair", stack.bwd_pair(li))]
-        else:
-            calls += [("gemm", c) for c in stack.gemm_calls(li)]
-        for kind, c in calls:
-            hold_stream(stream)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for _ in range(reps):
-                if kind == "quantize":
-                    fp8.fp8_quantize(*c, stream=stream)
-                elif kind == "pair":
-                    fp8.fp8_mm_grouped(c, stream=stream)
-                else:
-                    stack.mm(c, stream)
-            e1.record(stream)
-            e1.synchronize()
-            ms = e0.elapsed_time(e1) / reps
-            if kind == "quantize":
-                q_ms += ms
-                q_elems += c[1]
-                n_q += 1
-            elif kind == "pair":
-                g_ms += ms
-                f = sum(2 * M * N * K for (M, N, K) in (q[7:10] for q in c))
-                g_flops += f
-                g_bytes += sum(gemm_algorithmic_bytes(q[6], *q[7:10]) for q in c)
-                n_g += 1
-                per_shape[" + ".join(f"{'NT NN TN'.split()[q[6]]} {q[7]}x{q[8]}x{q[9]}" for q in c)] = (ms, f)
-            else:
-                M, N, K = c[7:10]
-                g_ms += ms
-                g_flops += 2 * M * N * K
-                g_bytes += gemm_algorithmic_bytes(c[6], M, N, K)
-                n_g += 1
-                per_shape[f"{'NT NN TN'.split()[c[6]]} {M}x{N}x{K}"] = (ms, 2 * M * N * K)
+    # stream, as inside the graph. The roofline figures rotate every call over
+    # copies of its inputs and outputs that together exceed twice the L2 (HBM
+    # traffic, as in the step, where a whole step's bytes pass between two uses
+    # of one tensor); the same calls on one L2-resident set are reported apart.
+    hot = breakdown(fp8, stack, stream, args.breakdown_reps, rotate=False)
+    cold = breakdown(fp8, stack, stream, args.breakdown_reps, rotate=True)
+    q_ms, q_elems, n_q = cold["q_ms"], cold["q_elems"], cold["n_q"]
+    g_ms, g_flops, g_bytes, n_g = cold["g_ms"], cold["g_flops"], cold["g_bytes"], cold["n_g"]
     # the grouped step-start launch (all W + the first x) against its
     # tensors quantized one launch each
     jobs = stack.grouped_call(0)
+    reps = args.breakdown_reps
     hold_stream(stream)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
@@ -478,11 +522,26 @@ def run_ours(args, world, rank, local):
     grouped_detail = {"jobs": len(jobs), "elems": many_elems, "us": round(1e3 * many_ms, 2),
                       "gbs": round(3.0 * many_elems / (many_ms * 1e-3) / 1e9, 1),
                       "frac": round(3.0 * many_elems / (many_ms * 1e-3) / 1e9 / hbm, 4),
-                      "same_tensors_one_launch_each_us": round(1e3 * single_ms, 2)}
+                      "same_tensors_one_launch_each_us": round(1e3 * single_ms, 2),
+                      "l2": "one input set (14.7 M elements, 29 MB bf16): L2-resident"}
     gemm_tf = g_flops / (g_ms * 1e-3) / 1e12
     quant_gbs = 3.0 * q_elems / (q_ms * 1e-3) / 1e9
-    gemm_detail = {k: {"us": round(1e3 * ms, 2), "tflops": round(f / (ms * 1e-3) / 1e12, 1)}
-                   for k, (ms, f) in per_shape.items()}
+    gemm_detail = {k: {"us": round(1e3 * ms, 2), "tflops": round(f / (ms * 1e-3) / 1e12, 1),
+                       "us_l2_hot": round(1e3 * hot["per_shape"][k][0], 2)}
+                   for k, (ms, f) in cold["per_shape"].items()}
+    quant_detail = {k: {"us": round(1e3 * ms, 2), "gbs": round(3.0 * n / (ms * 1e-3) / 1e9, 1),
+                        "us_l2_hot": round(1e3 * hot["per_tensor"][k][0], 2)}
+                    for k, (ms, n) in cold["per_tensor"].items()}
+    l2_hot = {"gemm_avg_launch_us": round(1e3 * hot["g_ms"] / hot["n_g"], 2),
+              "gemm_tflops": round(hot["g_flops"] / (hot["g_ms"] * 1e-3) / 1e12, 1),
+              "quantize_avg_launch_us": round(1e3 * hot["q_ms"] / hot["n_q"], 2),
+              "quantize_gbs": round(3.0 * hot["q_elems"] / (hot["q_ms"] * 1e-3) / 1e9, 1),
+              "method": "the same calls repeated on one input set (every tensor fits in the 126 MB L2)"}
+    configs = None
+    if not args.no_configs:
+        with ClockSampler(local) as cfg_clocks:
+            configs = run_configs(fp8, stream, hbm, fp8_burst)
+        configs["clocks"] = cfg_clocks.summary()
 
     # ---- e2e: host buffers through the public API ------------------------
     e2e = None
@@ -490,7 +549,10 @@ def run_ours(args, world, rank, local):
         e2e = run_e2e(fp8, stack, stream, args.e2e_steps, world, side, grouped)
         e2e["value"] = round(e2e["value"], 3)
 
-    context = {} if args.no_compare else compare_bf16(stack, ms_step, 200)
+    context = {}
+    if not args.no_compare:
+        context = compare_bf16(stack, ms_step, 200)
+        context["at_16384_tokens"] = compare_at_tokens(fp8, 8 * W.TOKENS, 50)
     gpu_launches = stack.launches_per_step(grouped) * args.steps
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
@@ -528,8 +590,13 @@ def run_ours(args, world, rank, local):
                               "peak_source": f"{peak_src} hbm copy",
                               "algorithmic_bytes_per_launch": round(3 * q_elems / n_q),
                               "avg_launch_us": round(1e3 * q_ms / n_q, 2)},
+        "breakdown_method": "each kernel repeated back to back, inputs and outputs rotating over copies that "
+                            "exceed 2x L2 (HBM reads, as in the step); us_l2_hot: the same on one set",
         "gemm_by_shape": gemm_detail,
+        "quantize_by_tensor": quant_detail,
+        "kernels_l2_hot": l2_hot,
         "quantize_grouped": grouped_detail,
+        "configs": configs,
         "clocks": clocks.summary(),
         "context": context,
         "e2e": e2e,
@@ -541,11 +608,11 @@ def run_ours(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
-def _rotated_graph_time(make_fn, reps, warm=3):
+def _rotated_graph_time(make_fn, reps, warm=3, n_sets=N_SETS):
     """One CUDA graph per input set, replayed in rotation over the sets, as
     the FP8 step is timed; ms per replay."""
     st = torch.cuda.Stream()
-    fns = [make_fn(s) for s in range(N_SETS)]
+    fns = [make_fn(s) for s in range(n_sets)]
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(side):
@@ -562,12 +629,12 @@ def _rotated_graph_time(make_fn, reps, warm=3):
         graphs.append(g)
     torch.cuda.synchronize()
     with torch.cuda.stream(st):
-        for i in range(warm * N_SETS):
-            graphs[i % N_SETS].replay()
+        for i in range(warm * n_sets):
+            graphs[i % n_sets].replay()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(st)
         for i in range(reps):
-            graphs[i % N_SETS].replay()
+            graphs[i % n_sets].replay()
         e1.record(st)
     e1.synchronize()
     ms = e0.elapsed_time(e1) / reps
@@ -585,7 +652,8 @@ def compare_bf16(stack, fp8_ms, reps):
     for the FP8-over-bf16 speed-up the AstrAI commit logs report for their
     kernels on L20."""
     out = {}
-    T = W.TOKENS
+    T = stack.tokens
+    n_sets = len(stack.sets)
     ys = [torch.empty(T, L["d_out"], dtype=torch.bfloat16, device="cuda") for L in stack.lin]
     dxs = [torch.empty(T, L["d_in"], dtype=torch.bfloat16, device="cuda") for L in stack.lin]
     dws = [torch.empty(L["d_out"], L["d_in"], dtype=torch.bfloat16, device="cuda") for L in stack.lin]
@@ -602,7 +670,7 @@ def compare_bf16(stack, fp8_ms, reps):
                 torch.matmul(t["g"].t(), t["x"], out=dws[li])
         return fn
 
-    bf16_ms = _rotated_graph_time(bf16_step, reps)
+    bf16_ms = _rotated_graph_time(bf16_step, reps, n_sets=n_sets)
     out["bf16_cublas_step_ms"] = round(bf16_ms, 4)
     out["fp8_over_bf16_step"] = round(bf16_ms / fp8_ms, 3)
 
@@ -612,7 +680,7 @@ def compare_bf16(stack, fp8_ms, reps):
         mods8 = [Fp8Linear(L["d_in"], L["d_out"], bias=False, device="cuda") for L in stack.lin]
         mods16 = [torch.nn.Linear(L["d_in"], L["d_out"], bias=False, device="cuda", dtype=torch.bfloat16)
                   for L in stack.lin]
-        xs = [[t["x"].detach().clone().requires_grad_(True) for t in stack.sets[s]] for s in range(N_SETS)]
+        xs = [[t["x"].detach().clone().requires_grad_(True) for t in stack.sets[s]] for s in range(n_sets)]
 
         def ag_step(mods):
             def make(s):
@@ -626,11 +694,31 @@ def compare_bf16(stack, fp8_ms, reps):
                 return fn
             return make
 
-        out["autograd_fp8_step_ms"] = round(_rotated_graph_time(ag_step(mods8), reps), 4)
-        out["autograd_bf16_step_ms"] = round(_rotated_graph_time(ag_step(mods16), reps), 4)
+        out["autograd_fp8_step_ms"] = round(_rotated_graph_time(ag_step(mods8), reps, n_sets=n_sets), 4)
+        out["autograd_bf16_step_ms"] = round(_rotated_graph_time(ag_step(mods16), reps, n_sets=n_sets), 4)
         out["autograd_fp8_over_bf16"] = round(out["autograd_bf16_step_ms"] / out["autograd_fp8_step_ms"], 3)
     except Exception as e:  # capture failures are reported, not hidden
         out["autograd_error"] = f"{type(e).__name__}: {e}"[:200]
+    return out
+
+
+def compare_at_tokens(fp8, tokens, reps):
+    """The FP8 step and its bf16 / autograd comparisons at a larger token
+    count: one input set (more than 2x L2 at 16384 tokens), the step as one
+    CUDA graph."""
+    stack = Stack(fp8, n_sets=1, tokens=tokens)
+    st = torch.cuda.Stream()
+    with torch.cuda.stream(st):
+        for _ in range(3):
+            stack.step(0, st, None, True)
+    torch.cuda.synchronize()
+    ms = _rotated_graph_time(lambda s: (lambda: stack.step(0, torch.cuda.current_stream(), None, True)), reps,
+                             n_sets=1)
+    out = {"tokens": tokens, "fp8_step_ms": round(ms, 4), "fp8_step_tflops": round(stack.flops / (ms * 1e-3) / 1e12, 1)}
+    out.update(compare_bf16(stack, ms, reps))
+    del stack
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
     return out
 
 
@@ -697,6 +785,185 @@ def run_e2e(fp8, stack, stream, steps, world, side=None, grouped=True):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": round(t_ms / steps, 3),
             "pipeline": "inputs and outputs double-buffered; H2D and D2H on two copy streams"}
+
+
+# ------------------------------------------------- the other workloads -----
+#
+# The workload table's other configurations, timed in the same run under the
+# same clock record: the NT 256^3 GEMM with bias, the square sweep in all
+# three layouts, the skinny shapes with bias, the batched shapes, and the
+# quantize size sweep. Every timed loop runs back to back on one stream held
+# in a device sleep while the host enqueues, and rotates over enough distinct
+# buffer sets that one pass over them is more than twice the L2, so every
+# launch reads its operands from HBM (the 256^3 case is 0.3 MB and stays
+# L2-resident: it is latency-bound and reported in microseconds).
+
+def _l2_bytes():
+    try:
+        return int(torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size)
+    except Exception:
+        return 126 << 20
+
+
+def _slots(set_bytes, cap=64):
+    """Buffer sets so that one rotation moves more than twice the L2."""
+    return int(min(cap, max(2, -(-2 * _l2_bytes() // max(1, set_bytes)))))
+
+
+def _time_us(stream, call, reps, warm=3):
+    """Device microseconds per call of call(i), i = 0 .. reps-1, back to back."""
+    with torch.cuda.stream(stream):
+        for i in range(warm):
+            call(i)
+    torch.cuda.synchronize()
+    hold_stream(stream, 500 + 40 * reps)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(reps):
+            call(warm + i)  # the rotation continues where the warm-up left it
+        e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) * 1e3 / reps
+
+
+def _gemm_entry(us, flops, nbytes, hbm, fp8_peak):
+    """One GEMM's line: time, TF/s and its fraction of the binding roof
+    (the slower of FLOPs at the FP8 peak and compulsory bytes at HBM)."""
+    t_tensor = flops / (fp8_peak * 1e12) * 1e6
+    t_hbm = nbytes / (hbm * 1e9) * 1e6
+    bound = "tensor" if t_tensor >= t_hbm else "hbm"
+    return {"us": round(us, 2), "tflops": round(flops / (us * 1e-6) / 1e12, 1),
+            "gbs": round(nbytes / (us * 1e-6) / 1e9, 1), "bound": bound,
+            "frac": round(max(t_tensor, t_hbm) / us, 4)}
+
+
+def run_configs(fp8, stream, hbm, fp8_peak, reps=20):
+    """Every workload of the table but the linear stack, timed on the device."""
+    dev = "cuda"
+    out = {"method": "back-to-back launches, CUDA events on the launching stream; buffers rotate over sets "
+                     "whose total is > 2x L2, so operands come from HBM (except the 0.3 MB NT 256^3)"}
+
+    def ring():
+        r = torch.empty(20, dtype=torch.int32, device=dev)
+        fp8.fp8_ring_init(r, 1.0)
+        return r
+
+    one = lambda v: torch.tensor([float(v)], device=dev)
+
+    # -- NT 256^3, A and B current-scaled to E4M3 from bf16, bf16 bias --------
+    M = N = K = 256
+    a = W.bf16_normal((M, K), 1.0, 1001).to(dev)
+    b = W.bf16_normal((N, K), 1.0, 1002).to(dev)
+    bias = W.bf16_normal((N,), 0.1, 1003).to(dev)
+    a8 = torch.empty(M * K, dtype=torch.uint8, device=dev)
+    b8 = torch.empty(N * K, dtype=torch.uint8, device=dev)
+    am, bm, sa, sb = (torch.empty(1, device=dev) for _ in range(4))
+    y = torch.empty(M * N, dtype=torch.bfloat16, device=dev)
+    qa = lambda i: fp8.fp8_quantize(a, M * K, E4M3, None, a8, am, sa, stream=stream)
+    qb = lambda i: fp8.fp8_quantize(b, N * K, E4M3, None, b8, bm, sb, stream=stream)
+    mm = lambda i: fp8.fp8_mm(a8, E4M3, b8, E4M3, sa, sb, NT, M, N, K, 1, 0, 0, 0, bias, None, 0, y, stream=stream)
+
+    def seq(i):
+        qa(i)
+        qb(i)
+        mm(i)
+    out["nt_256_bias_current"] = {
+        "us_quantize_a": round(_time_us(stream, qa, reps), 2), "us_gemm": round(_time_us(stream, mm, reps), 2),
+        "us_sequence": round(_time_us(stream, seq, reps), 2), "bound": "latency (0.03 GFLOP, 0.3 MB)",
+        "sequence": "current-scaled quantize of A and of B (each: amax pass + quantize pass), GEMM + bias"}
+
+    # -- square sweep on pre-quantized codes, NT / NN / TN ---------------------
+    sq = {}
+    for n in W.SQUARE_SIZES:
+        set_bytes = 2 * n * n + 2 * n * n
+        k = _slots(set_bytes)
+        ha = W.fp8_codes((n * n,), E4M3, 3000 + n)
+        hb = W.fp8_codes((n * n,), E4M3, 3100 + n)
+        sc = W.uniform(0.5, 2.0, 3200 + n, 2)
+        A = [ha.to(dev) for _ in range(k)]
+        B = [hb.to(dev) for _ in range(k)]
+        C = [torch.empty(n * n, dtype=torch.bfloat16, device=dev) for _ in range(k)]
+        s_a, s_b = one(sc[0]), one(sc[1])
+        r = 10 if n >= 8192 else reps
+        for lay, name in ((NT, "NT"), (NN, "NN"), (TN, "TN")):
+            call = lambda i, lay=lay: fp8.fp8_mm(A[i % k], E4M3, B[i % k], E4M3, s_a, s_b, lay, n, n, n, 1, 0, 0, 0,
+                                                  None, None, 0, C[i % k], stream=stream)
+            us = _time_us(stream, call, r)
+            e = _gemm_entry(us, 2.0 * n ** 3, gemm_algorithmic_bytes(lay, n, n, n), hbm, fp8_peak)
+            e["sets"] = k
+            sq[f"{name} {n}^3"] = e
+        del A, B, C
+    out["square"] = sq
+
+    # -- skinny / rectangular NT with bf16 bias, current-scaled operands -------
+    sk = {}
+    for (M, N, K) in W.SKINNY_SHAPES:
+        set_bytes = M * K + N * K + 2 * M * N
+        k = _slots(set_bytes)
+        xa = W.bf16_normal((M * K,), 1.0, 4000 + M).to(dev)
+        xb = W.bf16_normal((N * K,), 1.0, 4100 + N + K).to(dev)
+        bias = W.bf16_normal((N,), 0.1, 4200 + N).to(dev)
+        a8 = torch.empty(M * K, dtype=torch.uint8, device=dev)
+        b8 = torch.empty(N * K, dtype=torch.uint8, device=dev)
+        am, bm, s_a, s_b = (torch.empty(1, device=dev) for _ in range(4))
+        fp8.fp8_quantize(xa, M * K, E4M3, None, a8, am, s_a, stream=stream)
+        us_qb = _time_us(stream, lambda i: fp8.fp8_quantize(xb, N * K, E4M3, None, b8, bm, s_b, stream=stream), reps)
+        A = [a8.clone() for _ in range(k)]
+        B = [b8.clone() for _ in range(k)]
+        C = [torch.empty(M * N, dtype=torch.bfloat16, device=dev) for _ in range(k)]
+        call = lambda i: fp8.fp8_mm(A[i % k], E4M3, B[i % k], E4M3, s_a, s_b, NT, M, N, K, 1, 0, 0, 0, bias, None,
+                                     0, C[i % k], stream=stream)
+        us = _time_us(stream, call, reps)
+        e = _gemm_entry(us, 2.0 * M * N * K, gemm_algorithmic_bytes(NT, M, N, K) + 2 * N, hbm, fp8_peak)
+        e["sets"] = k
+        e["us_quantize_b_current"] = round(us_qb, 2)
+        sk[f"NT {M}x{N}x{K} +bias"] = e
+        del A, B, C
+    out["skinny"] = sk
+
+    # -- batched, per-tensor scales; the second case broadcasts B ---------------
+    bt = {}
+    for (batch, M, N, K, bcast) in W.BATCHED:
+        nb = 1 if bcast else batch
+        set_bytes = batch * M * K + nb * N * K + 2 * batch * M * N
+        k = _slots(set_bytes)
+        ha = W.fp8_codes((batch * M * K,), E4M3, 5000 + batch)
+        hb = W.fp8_codes((nb * N * K,), E4M3, 5100 + batch)
+        A = [ha.to(dev) for _ in range(k)]
+        B = [hb.to(dev) for _ in range(k)]
+        C = [torch.empty(batch * M * N, dtype=torch.bfloat16, device=dev) for _ in range(k)]
+        s_a, s_b = one(0.75), one(1.5)
+        sbt = 0 if bcast else N * K
+        call = lambda i: fp8.fp8_mm(A[i % k], E4M3, B[i % k], E4M3, s_a, s_b, NT, M, N, K, batch, M * K, sbt, M * N,
+                                     None, None, 0, C[i % k], stream=stream)
+        us = _time_us(stream, call, reps)
+        e = _gemm_entry(us, 2.0 * batch * M * N * K, set_bytes, hbm, fp8_peak)
+        e["sets"] = k
+        bt[f"{batch}x{M}x{N}x{K}" + (" B stride 0" if bcast else "")] = e
+        del A, B, C
+    out["batched"] = bt
+
+    # -- quantize sweep: delayed E4M3, 3 B per element --------------------------
+    qs = {}
+    base = W.bf16_normal((1 << 24,), 1.0, 6001).to(dev)
+    for lg in (22, 24, 26, 28):
+        n = 1 << lg
+        k = _slots(3 * n)
+        reps_q = max(reps, k)
+        X = [base[:n].clone() if n <= base.numel() else base.repeat(n // base.numel()) for _ in range(k)]
+        Q = [torch.empty(n, dtype=torch.uint8, device=dev) for _ in range(k)]
+        rg = ring()
+        am, sc = torch.empty(1, device=dev), torch.empty(1, device=dev)
+        call = lambda i: fp8.fp8_quantize(X[i % k], n, E4M3, rg, Q[i % k], am, sc, stream=stream)
+        us = _time_us(stream, call, reps_q)
+        gbs = 3.0 * n / (us * 1e-6) / 1e9
+        qs[f"2^{lg}"] = {"us": round(us, 2), "gbs": round(gbs, 1), "frac": round(gbs / hbm, 4), "sets": k}
+        del X, Q
+    out["quantize_delayed_e4m3"] = qs
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
 
 
 # ------------------------------------------------------- the CPU oracle -----
@@ -895,12 +1162,13 @@ def run_kernel(args):
     torch.cuda.synchronize()
     hold_stream(st)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(st):
-        e0.record(st)
-        for i in range(reps):
-            call(i)
-        e1.record(st)
-    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        with torch.cuda.stream(st):
+            e0.record(st)
+            for i in range(reps):
+                call(i)
+            e1.record(st)
+        torch.cuda.synchronize()
     us = e0.elapsed_time(e1) * 1e3 / reps
     if args.kernel in ("gemm", "cublaslt", "bwd_pair"):
         ach = units / (us * 1e-6) / 1e12
@@ -909,12 +1177,13 @@ def run_kernel(args):
                           "layout": {"gemm": args.layout, "cublaslt": "NT", "bwd_pair": "NN + TN"}[args.kernel],
                           "us": round(us, 2),
                           "tflops": round(ach, 1), "frac_fp8_peak": round(ach / peak, 4), "peak": peak,
-                          "peak_source": src}))
+                          "peak_source": src, "clocks": clocks.summary()}))
     else:
         ach = units / (us * 1e-6) / 1e9
         n_el = int(units / 4) if args.kernel == "quantize_2d" else int(units / 3)
         print(json.dumps({"kernel": args.kernel, "n": n_el, "us": round(us, 2), "gbs": round(ach, 1),
-                          "frac_hbm": round(ach / hbm, 4), "peak": hbm, "peak_source": src}))
+                          "frac_hbm": round(ach / hbm, 4), "peak": hbm, "peak_source": src,
+                          "clocks": clocks.summary()}))
 
 
 def main():
@@ -934,6 +1203,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-compare", action="store_true", help="skip the bf16 / autograd comparison")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other workloads (NT 256^3, square sweep, skinny, batched, quantize sweep)")
     ap.add_argument("--breakdown-reps", type=int, default=20)
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--kernel", choices=["gemm", "bwd_pair", "quantize", "quantize_many", "quantize_2d", "cublaslt"],

@@ -1456,12 +1456,39 @@ extern "C" size_t fp8_mm_workspace_size(int64_t M, int64_t N, int64_t K, int64_t
     return split_ws_bytes(tile_count(M, N, batch, tc.pair, tc.bn), tc.pair ? 2 : 1, tc.bn, tc.split);
 }
 
-// Library-owned split-K scratch for fp8_mm_splitk_static: the counters (zero
-// from module load, left zero by every completed call) and the fp32 partial
-// tiles, so that a split GEMM needs no allocation from the caller or the
-// library.
+// Library-owned split-K scratch for fp8_mm_splitk_static: the counter block
+// (kSplitCntBytes) followed by the fp32 partial tiles. One array per device
+// that loads the library, held until the process exits, shared by every call
+// on that device. Host code may not use the symbol itself as a pointer: on
+// the host it names a stand-in, not device memory, so the device address is
+// looked up once per device (scratch_address) and passed to the kernel.
 constexpr size_t kStaticScratchBytes = size_t(32) << 20;
 __device__ __align__(256) uint8_t g_splitk_scratch[kStaticScratchBytes];
+
+namespace fp8lite {
+namespace {
+
+// The scratch's device address on the current device, looked up on the first
+// call made with that device current and kept for later calls. The lookup may
+// load the library's GEMM module on that device, which stream capture does not
+// allow: the first call on a device must come before any capture.
+void* scratch_address() {
+    constexpr int kMaxDevices = 64;
+    static void* addr[kMaxDevices] = {};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_splitk_scratch) != cudaSuccess) return nullptr;
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
+}  // namespace
+}  // namespace fp8lite
 
 extern "C" fp8_status fp8_mm_splitk_static(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8, fp8_fmt fb,
                                            const float* sa, const float* sb, fp8_layout layout, int64_t M, int64_t N,
@@ -1471,8 +1498,14 @@ extern "C" fp8_status fp8_mm_splitk_static(const uint8_t* a8, fp8_fmt fa, const 
     if (split_k < 2 || split_k > kMaxSplit) return FP8_ERR_INVALID_ARG;
     const size_t need = fp8_mm_workspace_size(M, N, K, batch, layout, split_k);
     if (need > kStaticScratchBytes) return FP8_ERR_UNSUPPORTED;
-    void* scratch = nullptr;
-    if (cudaGetSymbolAddress(&scratch, g_splitk_scratch) != cudaSuccess) return FP8_ERR_CUDA;
+    void* scratch = scratch_address();
+    if (!scratch) return FP8_ERR_CUDA;
+    // The counters must be zero when the GEMM starts. A completed call leaves
+    // them zero, but a call whose bounded wait gave up may not; clearing them
+    // on the caller's stream makes every call start clean. The partial tiles
+    // need no clearing: each is written before it is read.
+    if (need > 0 && cudaMemsetAsync(scratch, 0, kSplitCntBytes, as_stream(stream)) != cudaSuccess)
+        return FP8_ERR_CUDA;
     // fp8_mm_ws validates the rest (and reports a split the problem cannot take)
     return fp8_mm_ws(a8, fa, b8, fb, sa, sb, layout, M, N, K, batch, stride_a, stride_b, stride_c, bias, bias_scale,
                      bias_fmt, out, scratch, kStaticScratchBytes, split_k, stream);

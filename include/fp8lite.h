@@ -337,15 +337,36 @@ FP8LITE_API fp8_status fp8_mm_out8(const uint8_t* a8, fp8_fmt fa, const uint8_t*
 FP8LITE_API size_t fp8_mm_workspace_size(int64_t M, int64_t N, int64_t K, int64_t batch, fp8_layout layout,
                                          int32_t split_k);
 
-/* fp8_mm_ws with split_k = 2 .. 4 on scratch the library owns: a 32 MiB
- * device array of the library (zero from load, its counters left zero by
- * every completed call), so the call allocates nothing and needs no
- * workspace from the caller. Same result, bit for bit, as fp8_mm_ws with the
- * same split_k. The scratch is one per device: calls that may run at the same
- * time on one device (e.g. on two streams) must not use this entry point.
+/* fp8_mm_ws with split_k = 2 .. 4, for callers that cannot allocate device
+ * memory. The pages have no counterpart: it is an addition of this library.
+ *
+ * Who needs it: code that runs where cudaMalloc is not available or not
+ * allowed -- a custom allocator or memory pool that owns every device byte,
+ * a plug-in or callback invoked from inside another framework's step, a
+ * real-time or embedded caller that may not allocate after start-up. Such a
+ * caller has no way to provide fp8_mm_ws's workspace. This entry point
+ * allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ * Its scratch is a 32 MiB device array of the library (a static device
+ * variable): every GPU that loads the library holds it until the process
+ * exits. The caller still passes the inputs and the output.
+ *
+ * Set-up: the first call on a device (with that device current) looks up the
+ * array's device address and keeps it; that lookup may load the library's
+ * GEMM module, which stream capture does not allow, so make the first call
+ * on each device outside any capture.
+ * Contents: every call on a device shares the array, which keeps the last
+ * call's contents. Each call first clears the array's 4096-byte counter block
+ * on `stream` (one cudaMemsetAsync; also after a call whose bounded wait gave
+ * up), and the fp32 partial tiles are written before they are read, so no
+ * state carries from one call into the next. Calls whose work overlaps on the
+ * GPU (two streams, or two host threads, on one device) race on the array and
+ * give undefined results: run them in order on one stream.
+ * Result: bit for bit what fp8_mm_ws gives with the same split_k.
  * Errors: as fp8_mm_ws; FP8_ERR_INVALID_ARG for split_k outside 2 .. 4;
- * FP8_ERR_UNSUPPORTED when the split needs more than the 32 MiB
- * (fp8_mm_workspace_size() > 33554432) or the problem cannot take it. */
+ * FP8_ERR_UNSUPPORTED when the split needs more scratch than the 32 MiB the
+ * library holds (fp8_mm_workspace_size(..., split_k) > 33554432) or the
+ * problem cannot take the split; FP8_ERR_CUDA if the address lookup or the
+ * clear fails. */
 FP8LITE_API fp8_status fp8_mm_splitk_static(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8, fp8_fmt fb,
                   const float* sa, const float* sb, fp8_layout layout,
                   int64_t M, int64_t N, int64_t K, int64_t batch,
@@ -388,7 +409,11 @@ FP8LITE_API fp8_status fp8_mm_grouped(const fp8_mm_problem* problems, int32_t co
 /* Synchronises the current device, then reads and clears the library's
  * device error word: FP8_ERR_DEVICE_TIMEOUT if a GEMM thread block gave up a
  * bounded wait since the last call (its output tile is then undefined),
- * FP8_OK otherwise, FP8_ERR_CUDA if the synchronisation failed. */
+ * FP8_OK otherwise, FP8_ERR_CUDA if the synchronisation failed.
+ * A diagnostic, not a hot-path call: it waits for all work on the device
+ * (every stream) and cannot be captured into a CUDA graph. After a timeout,
+ * a caller-owned split-K workspace (fp8_mm_ws) must be zeroed again before
+ * its next use; fp8_mm_splitk_static clears its own counters every call. */
 FP8LITE_API fp8_status fp8_last_device_error(void);
 
 /* Bias gradient of a linear layer: out[j] = bf16_rne( sum_i g[i][j] ), the

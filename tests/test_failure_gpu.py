@@ -29,6 +29,18 @@ def test_bounded_wait_times_out_cleanly():
     y, sums = oracle.mm(a8.numpy(), 0, b8.numpy(), 0, 1.0, 1.0, oracle.NT, 128, 128, 128)
     got = out.float().cpu().numpy().reshape(1, 128, 128)
     assert np.all(np.abs(got - y) <= oracle.tolerance(y, sums))
+    # a split-K call on the library's own scratch right after the timeout
+    # gives what the caller-workspace call gives, bit for bit
+    M, N, K = 2048, 1024, 4096
+    a8 = W.fp8_codes((M * K,), 0, 3).cuda()
+    b8 = W.fp8_codes((N * K,), 0, 4).cuda()
+    args = (a8, 0, b8, 0, s, s, fp8.FP8_NT, M, N, K, 1, 0, 0, 0, None, None, 0)
+    want = torch.empty(M * N, dtype=torch.bfloat16, device="cuda")
+    fp8.fp8_mm_ws(*args, want, g.workspace(fp8.fp8_mm_workspace_size(M, N, K, 1, fp8.FP8_NT, 2)), 2)
+    got = torch.empty_like(want)
+    fp8.fp8_mm_splitk_static(*args, got, 2)
+    torch.cuda.synchronize()
+    assert torch.equal(got.view(torch.int16), want.view(torch.int16))
     fp8.fp8_last_device_error()
 
 
