@@ -151,6 +151,22 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint
     }
 }
 
+// wait_bounded by every lane of a warp, with one verdict for all of them.
+__device__ __forceinline__ bool wait_bounded_warp(uint32_t bar, uint32_t parity) {
+    return __all_sync(0xffffffffu, wait_bounded(bar, parity));
+}
+
+// True in one lane of the (fully active) warp.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r));
+    return r != 0;
+}
+
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* ptr) {
     uint32_t v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
@@ -379,44 +395,47 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer ---
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            for (int i = 0, u = unit0; u < total_units && ok; u = unit_of<GROUP>(++i, unit0, unit_step)) {
-                int t = u / split;
-                const CUtensorMap* map_a = &tm_a;
-                const CUtensorMap* map_b = &tm_b;
-                bool a_mn = A_MN, b_mn = B_MN;
-                TileWalk w = walk;
-                int kbs = k_blocks;
-                int ebn = BN, n_base = 0;  // the unit's tile width and first column
-                if constexpr (GROUP) {
-                    const GroupProblem& q = group_problem(grp, u, t);
-                    map_a = &q.ta;
-                    map_b = &q.tb;
-                    a_mn = q.a_mn;
-                    b_mn = q.b_mn;
-                    w = {q.m_tiles, q.n_tiles, walk.group_m};
-                    kbs = q.k_blocks;
-                    ebn = q.bn;
-                    n_base = q.n_base;
-                }
-                const int kb0 = GROUP ? 0 : (u - t * split) * kb_per;
-                const int kb1 = GROUP ? kbs : min(k_blocks, kb0 + kb_per);
-                int mb, nb, b;
-                tile_coords(t, w, mb, nb, b);
-                const int ba = a_bcast ? 0 : b;
-                const int bb = b_bcast ? 0 : b;
-                const int m0 = mb * BM * CTAS + int(rank) * BM;
-                const int n0 = n_base + nb * ebn + int(rank) * (BN / CTAS);
-                const uint32_t stage_tx = GROUP ? uint32_t(L::kABytes + ebn * BK) : uint32_t(L::kStageTx);
-                for (int kb = kb0; kb < kb1; ++kb) {
-                    if (!wait_bounded(bar_empty + 8 * stage, phase ^ 1)) { ok = false; break; }
-                    const uint32_t full = bar_full + 8 * stage;
+        // The whole warp walks the units and waits on the barriers, so the
+        // loop's values stay warp-uniform; one elected lane issues the loads.
+        const bool issuer = elect_one();
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int i = 0, u = unit0; u < total_units && ok; u = unit_of<GROUP>(++i, unit0, unit_step)) {
+            int t = u / split;
+            const CUtensorMap* map_a = &tm_a;
+            const CUtensorMap* map_b = &tm_b;
+            bool a_mn = A_MN, b_mn = B_MN;
+            TileWalk w = walk;
+            int kbs = k_blocks;
+            int ebn = BN, n_base = 0;  // the unit's tile width and first column
+            if constexpr (GROUP) {
+                const GroupProblem& q = group_problem(grp, u, t);
+                map_a = &q.ta;
+                map_b = &q.tb;
+                a_mn = q.a_mn;
+                b_mn = q.b_mn;
+                w = {q.m_tiles, q.n_tiles, walk.group_m};
+                kbs = q.k_blocks;
+                ebn = q.bn;
+                n_base = q.n_base;
+            }
+            const int kb0 = GROUP ? 0 : (u - t * split) * kb_per;
+            const int kb1 = GROUP ? kbs : min(k_blocks, kb0 + kb_per);
+            int mb, nb, b;
+            tile_coords(t, w, mb, nb, b);
+            const int ba = a_bcast ? 0 : b;
+            const int bb = b_bcast ? 0 : b;
+            const int m0 = mb * BM * CTAS + int(rank) * BM;
+            const int n0 = n_base + nb * ebn + int(rank) * (BN / CTAS);
+            const uint32_t stage_tx = GROUP ? uint32_t(L::kABytes + ebn * BK) : uint32_t(L::kStageTx);
+            for (int kb = kb0; kb < kb1; ++kb) {
+                if (!wait_bounded_warp(bar_empty + 8 * stage, phase ^ 1)) { ok = false; break; }
+                const uint32_t full = bar_full + 8 * stage;
+                const uint32_t da = s_a + stage * L::kABytes;
+                const uint32_t db = s_b + stage * L::kBBytes;
+                if (issuer) {
                     if (leader) mbar_arrive_expect_tx(full, stage_tx);
-                    const uint32_t da = s_a + stage * L::kABytes;
-                    const uint32_t db = s_b + stage * L::kBBytes;
                     if (CTAS == 1) {
                         if (a_mn) tma_load_3d(da, map_a, full, m0, kb * BK, ba);
                         else      tma_load_3d(da, map_a, full, kb * BK, m0, ba);
@@ -434,18 +453,23 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                         if (B_MN) tma_load_3d_pair(db, &tm_b, lfull, n0, kb * BK, bb);
                         else      tma_load_3d_pair(db, &tm_b, lfull, kb * BK, n0, bb);
                     }
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
-            }
-            // drain: wait until the MMAs released every stage still in use
-            for (int i = 0; i < STAGES && ok; ++i) {
-                if (!wait_bounded(bar_empty + 8 * stage, phase ^ 1)) break;
+                __syncwarp();
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
         }
+        // drain: wait until the MMAs released every stage still in use
+        for (int i = 0; i < STAGES && ok; ++i) {
+            if (!wait_bounded_warp(bar_empty + 8 * stage, phase ^ 1)) break;
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
     } else if (warp == 1) {
         // --------------------------------------------------- MMA issuer ---
-        if (lane == 0 && leader) {
+        // As the producer: the warp walks and waits together, one elected
+        // lane issues every MMA and commit (a commit tracks the MMAs of the
+        // thread that issues it, so it is always the same lane).
+        const bool issuer = elect_one();
+        if (leader) {
             int stage = 0;
             uint32_t phase = 0;
             int it = 0;
@@ -466,17 +490,18 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                 const int kb1 = GROUP ? kbs : min(k_blocks, kb0 + kb_per);
                 const int buf = it & 1;
                 const uint32_t acc_phase = (it >> 1) & 1;
-                if (!wait_bounded(bar_tempty + 8 * buf, acc_phase ^ 1)) break;
+                if (!wait_bounded_warp(bar_tempty + 8 * buf, acc_phase ^ 1)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + buf * BN;
                 const uint64_t a_desc0 = a_mn ? smem_desc_sw128(s_a, 128 * BK, 1024) : smem_desc_sw128(s_a, 16, 1024);
                 const uint64_t b_desc0 = b_mn ? smem_desc_sw128(s_b, 128 * BK, 1024) : smem_desc_sw128(s_b, 16, 1024);
+                const uint64_t a_step = a_mn ? 256u : 2u, b_step = b_mn ? 256u : 2u;
                 for (int kb = kb0; kb < kb1; ++kb) {
                     // the stage's operands arrive through the async proxy and
                     // complete on this barrier: the MMAs may read them without
                     // a tcgen05 fence (that is needed only after the epilogue's
                     // hand-back of the accumulator, above)
-                    if (!wait_bounded(bar_full + 8 * stage, phase)) { ok = false; break; }
+                    if (!wait_bounded_warp(bar_full + 8 * stage, phase)) { ok = false; break; }
                     // the stage's descriptors: stage 0's plus the stage offset in
                     // the start-address field (16-byte units; no carry out of it,
                     // shared memory is below 256 KB). Each next 32-deep K slice is
@@ -484,15 +509,20 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                     // 128 bytes further (MN-major).
                     const uint64_t adesc = a_desc0 + uint64_t(stage) * (L::kABytes >> 4);
                     const uint64_t bdesc = b_desc0 + uint64_t(stage) * (L::kBBytes >> 4);
-                    mma_kblock_f8f6f4<CTAS>(d_tmem, adesc, bdesc, a_mn ? 256u : 2u, b_mn ? 256u : 2u, id,
-                                            kb != kb0);
-                    // release the stage (in both CTAs of a pair)
-                    if (CTAS == 1) mma_commit(bar_empty + 8 * stage);
-                    else           mma_commit_pair(bar_empty + 8 * stage);
+                    if (issuer) {
+                        mma_kblock_f8f6f4<CTAS>(d_tmem, adesc, bdesc, a_step, b_step, id, kb != kb0);
+                        // release the stage (in both CTAs of a pair)
+                        if (CTAS == 1) mma_commit(bar_empty + 8 * stage);
+                        else           mma_commit_pair(bar_empty + 8 * stage);
+                    }
+                    __syncwarp();
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
-                if (CTAS == 1) mma_commit(bar_tfull + 8 * buf);
-                else           mma_commit_pair(bar_tfull + 8 * buf);
+                if (issuer) {
+                    if (CTAS == 1) mma_commit(bar_tfull + 8 * buf);
+                    else           mma_commit_pair(bar_tfull + 8 * buf);
+                }
+                __syncwarp();
             }
         }
     } else {
