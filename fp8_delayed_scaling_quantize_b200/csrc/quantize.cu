@@ -458,12 +458,46 @@ int sm_count() {
     return cached[dev];
 }
 
+// Blocks of a single-tensor launch. Every block adds its amax and takes a
+// ticket on the ring's one cache line, and those same-address atomics queue
+// (about 2 ns each on B200), so below 64 M elements the grid is kept at one
+// to two blocks per SM: at least one per SM, so that every SM's loads are in
+// flight (as long as each thread still gets a unit), and at most two, each
+// thread looping over further rounds of kUnroll units. From 64 M elements on
+// the atomics are a small part of the time and four blocks per SM keep more
+// loads in flight. Measured on B200 (delayed E4M3, back-to-back launches,
+// microseconds, grid of up to four blocks per SM -> this one): 1M elements
+// 3.81 -> 3.52, 2M 3.81 -> 3.73, 8M 7.04 -> 5.65, 16M 10.63 -> 9.48; 256M
+// elements took 125.8 with four blocks per SM and 129.9 with two.
 int grid_for(int64_t n) {
     const int64_t units = n >> 3;
+    const int64_t sms = sm_count();
     const int64_t want = (units + int64_t(kThreads) * kUnroll - 1) / (int64_t(kThreads) * kUnroll);
-    const int64_t cap = int64_t(sm_count()) * (2048 / kThreads);
-    int64_t g = want < cap ? want : cap;
+    const int64_t busy = (units + kThreads - 1) / kThreads;  // blocks whose every thread has a unit
+    const int64_t cap = (n >= (int64_t(1) << 26) ? 4 : 2) * sms;
+    int64_t g = want < sms ? sms : want;
+    if (g > cap) g = cap;
+    if (g > busy) g = busy;
     return int(g < 1 ? 1 : g);
+}
+
+// Blocks of each job of a grouped launch: the whole launch gets the blocks
+// one large tensor would (two per SM), shared in proportion to the jobs'
+// sizes, each job at least one block and at most one unit per thread. Every
+// job's atomics go to its own ring, so fewer blocks in all means less
+// queueing on each ring's line. Measured on B200 on the linear stack's
+// step-start launch (every weight and the first activation, 14.7 M elements,
+// microseconds): each job sized as its own launch 9.46, in proportion 8.93.
+void grid_many(const fp8_quantize_job* jobs, int count, int* blocks) {
+    int64_t all = 0;
+    for (int j = 0; j < count; ++j) all += jobs[j].n;
+    const int64_t budget = 2 * int64_t(sm_count());
+    for (int j = 0; j < count; ++j) {
+        const int64_t share = all > 0 ? (budget * jobs[j].n + all - 1) / all : 1;
+        const int64_t busy = ((jobs[j].n >> 3) + kThreads - 1) / kThreads;
+        const int64_t g = share < busy ? share : busy;
+        blocks[j] = int(g < 1 ? 1 : g);
+    }
 }
 
 template <int FMT, int IN>
@@ -668,6 +702,10 @@ extern "C" fp8_status fp8_quantize_many_ex(const fp8_quantize_job* jobs, int32_t
     QuantJobs q = {};
     q.count = count;
     int total = 0;
+    for (int j = 0; j < count; ++j)  // sizes first: the grid is shared in proportion to them
+        if (jobs[j].n < 0 || jobs[j].n >= (int64_t(1) << 40)) return FP8_ERR_INVALID_ARG;
+    int blocks[FP8_QUANTIZE_MAX_JOBS];
+    grid_many(jobs, count, blocks);
     for (int j = 0; j < count; ++j) {
         const fp8_quantize_job& in = jobs[j];
         if (!valid_fmt(in.fmt) || !valid_dtype(in.dtype)) return FP8_ERR_INVALID_ARG;
@@ -679,7 +717,7 @@ extern "C" fp8_status fp8_quantize_many_ex(const fp8_quantize_job* jobs, int32_t
         for (int k = 0; k < j; ++k)
             if (jobs[k].ring == in.ring) return FP8_ERR_INVALID_ARG;  // one ring, one call at a time
         q.first[j] = total;
-        q.blocks[j] = grid_for(in.n);
+        q.blocks[j] = blocks[j];
         total += q.blocks[j];
         q.fmt[j] = int(in.fmt);
         q.dtype[j] = int(in.dtype);
