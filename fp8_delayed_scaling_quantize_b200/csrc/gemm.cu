@@ -303,6 +303,36 @@ __device__ __forceinline__ bool epilogue_bar_or(bool v) {
     return r != 0;
 }
 
+// One 128 x 32 bf16 block of the epilogue: to the staging tile whose last
+// store is known to have read it (64-byte swizzle: 16-byte piece j of row r at
+// (j ^ (r / 2 mod 4)) * 16, so the 8 lanes of a store phase hit distinct
+// banks), then one TMA store by the lead thread, which clips the M / N tails
+// of the output. n_st counts the stores issued so far (they take the staging
+// tiles in turn).
+template <typename L>
+__device__ __forceinline__ void stage_and_store(uint32_t stg0, int n_st, int row_in_tile, const float (&y)[32],
+                                                bool store_lead, const CUtensorMap* map_c, int col0, int m0, int b) {
+    const uint32_t stg = stg0 + uint32_t(n_st % L::kStgBufs) * L::kStgBytes;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t addr = stg + row_in_tile * 64 + ((j ^ ((row_in_tile >> 1) & 3)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pack_bf16x2(y[8 * j + 0], y[8 * j + 1])),
+                     "r"(pack_bf16x2(y[8 * j + 2], y[8 * j + 3])), "r"(pack_bf16x2(y[8 * j + 4], y[8 * j + 5])),
+                     "r"(pack_bf16x2(y[8 * j + 6], y[8 * j + 7]))
+                     : "memory");
+    }
+    fence_proxy_async_smem();
+    // the store two blocks back has read its tile, which the next block
+    // reuses (only the newest store may still be reading); the barrier
+    // publishes that and this block
+    if (store_lead) bulk_wait_read<L::kStgBufs - 2>();
+    epilogue_bar();
+    if (store_lead) {
+        tma_store_3d(map_c, stg, col0, m0, b);
+        bulk_commit();
+    }
+}
+
 // One kernel for both tile shapes: CTAS = 1 computes 128 x BN tiles per CTA;
 // CTAS = 2 runs as clusters of two CTAs on two SMs computing 256 x BN tiles
 // with tcgen05 cta_group::2 -- the leader issues the MMAs, each CTA loads its
@@ -389,46 +419,69 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     // The prologue above overlaps the previous kernel's tail; operands,
-    // scales and the output are touched only after it has completed.
-    griddep_wait();
-    griddep_launch();
+    // scales and the output are touched only after it has completed. Each
+    // role waits for it separately, so that the producer can work out its
+    // first unit's tile (pure arithmetic on the parameters) before.
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer ---
         // The whole warp walks the units and waits on the barriers, so the
         // loop's values stay warp-uniform; one elected lane issues the loads.
         const bool issuer = elect_one();
+        struct Plan {
+            const CUtensorMap* map_a;
+            const CUtensorMap* map_b;
+            int kb0, kb1, m0, n0, ba, bb, ebn;
+            uint32_t stage_tx;
+            bool a_mn, b_mn;
+        };
+        // the loads of work unit u: maps, k-block range, tile origin, batch
+        auto plan = [&](int u) {
+            Plan pl;
+            int t = u / split;
+            pl.map_a = &tm_a;
+            pl.map_b = &tm_b;
+            pl.a_mn = A_MN;
+            pl.b_mn = B_MN;
+            TileWalk w = walk;
+            int kbs = k_blocks;
+            int n_base = 0;
+            pl.ebn = BN;  // the unit's tile width
+            if constexpr (GROUP) {
+                const GroupProblem& q = group_problem(grp, u, t);
+                pl.map_a = &q.ta;
+                pl.map_b = &q.tb;
+                pl.a_mn = q.a_mn;
+                pl.b_mn = q.b_mn;
+                w = {q.m_tiles, q.n_tiles, walk.group_m};
+                kbs = q.k_blocks;
+                pl.ebn = q.bn;
+                n_base = q.n_base;
+            }
+            pl.kb0 = GROUP ? 0 : (u - t * split) * kb_per;
+            pl.kb1 = GROUP ? kbs : min(k_blocks, pl.kb0 + kb_per);
+            int mb, nb, b;
+            tile_coords(t, w, mb, nb, b);
+            pl.ba = a_bcast ? 0 : b;
+            pl.bb = b_bcast ? 0 : b;
+            pl.m0 = mb * BM * CTAS + int(rank) * BM;
+            pl.n0 = n_base + nb * pl.ebn + int(rank) * (BN / CTAS);
+            pl.stage_tx = GROUP ? uint32_t(L::kABytes + pl.ebn * BK) : uint32_t(L::kStageTx);
+            return pl;
+        };
+        Plan pl = {};
+        if (unit0 < total_units) pl = plan(unit0);  // before the wait: it reads no memory
+        griddep_wait();
+        griddep_launch();
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
-        for (int i = 0, u = unit0; u < total_units && ok; u = unit_of<GROUP>(++i, unit0, unit_step)) {
-            int t = u / split;
-            const CUtensorMap* map_a = &tm_a;
-            const CUtensorMap* map_b = &tm_b;
-            bool a_mn = A_MN, b_mn = B_MN;
-            TileWalk w = walk;
-            int kbs = k_blocks;
-            int ebn = BN, n_base = 0;  // the unit's tile width and first column
-            if constexpr (GROUP) {
-                const GroupProblem& q = group_problem(grp, u, t);
-                map_a = &q.ta;
-                map_b = &q.tb;
-                a_mn = q.a_mn;
-                b_mn = q.b_mn;
-                w = {q.m_tiles, q.n_tiles, walk.group_m};
-                kbs = q.k_blocks;
-                ebn = q.bn;
-                n_base = q.n_base;
-            }
-            const int kb0 = GROUP ? 0 : (u - t * split) * kb_per;
-            const int kb1 = GROUP ? kbs : min(k_blocks, kb0 + kb_per);
-            int mb, nb, b;
-            tile_coords(t, w, mb, nb, b);
-            const int ba = a_bcast ? 0 : b;
-            const int bb = b_bcast ? 0 : b;
-            const int m0 = mb * BM * CTAS + int(rank) * BM;
-            const int n0 = n_base + nb * ebn + int(rank) * (BN / CTAS);
-            const uint32_t stage_tx = GROUP ? uint32_t(L::kABytes + ebn * BK) : uint32_t(L::kStageTx);
+        for (int i = 0, u = unit0; u < total_units && ok;) {
+            const CUtensorMap* map_a = pl.map_a;
+            const CUtensorMap* map_b = pl.map_b;
+            const bool a_mn = pl.a_mn, b_mn = pl.b_mn;
+            const int kb0 = pl.kb0, kb1 = pl.kb1, m0 = pl.m0, n0 = pl.n0, ba = pl.ba, bb = pl.bb, ebn = pl.ebn;
+            const uint32_t stage_tx = pl.stage_tx;
             for (int kb = kb0; kb < kb1; ++kb) {
                 if (!wait_bounded_warp(bar_empty + 8 * stage, phase ^ 1)) { ok = false; break; }
                 const uint32_t full = bar_full + 8 * stage;
@@ -457,6 +510,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                 __syncwarp();
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
+            u = unit_of<GROUP>(++i, unit0, unit_step);
+            if (u < total_units) pl = plan(u);
         }
         // drain: wait until the MMAs released every stage still in use
         for (int i = 0; i < STAGES && ok; ++i) {
@@ -465,6 +520,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         }
     } else if (warp == 1) {
         // --------------------------------------------------- MMA issuer ---
+        griddep_wait();
+        griddep_launch();
         // As the producer: the warp walks and waits together, one elected
         // lane issues every MMA and commit (a commit tracks the MMAs of the
         // thread that issues it, so it is always the same lane).
@@ -527,6 +584,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         }
     } else {
         // ----------------------------------------------------- epilogue ---
+        griddep_wait();
+        griddep_launch();
         const int q = warp & 3;             // TMEM lane quarter this warp may access
         const int row_in_tile = q * 32 + lane;
         const int etid = threadIdx.x - 64;  // 0 .. kEpiThreads-1
@@ -657,6 +716,46 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             }
             uint16_t* orow = SWAP ? out_base + int64_t(b) * p.stride_c + row
                                   : out_base + int64_t(b) * p.stride_c + int64_t(row) * N;
+            if constexpr (!SPLIT && !SWAP && !OUT8) {
+                if (tma_store) {
+                    // The common case, pipelined: chunk c + 1's accumulator
+                    // columns leave TMEM while chunk c is converted, staged and
+                    // stored (two register sets, the wait tied to the set it
+                    // waits for).
+                    const int col_first = n_base + nb * ebn;
+                    const int left = (N - col_first + 31) / 32;
+                    const int nch = left < ebn / 32 ? left : ebn / 32;
+                    auto emit = [&](const uint32_t (&r)[32], int c) {
+                        float y[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const float bias = HAS_BIAS ? s_bias[c * 32 + i] : 0.0f;
+                            y[i] = fmaf(__uint_as_float(r[i]), inv, bias);
+                        }
+                        stage_and_store<L>(stg0, n_st, row_in_tile, y, store_lead, map_c, col_first + c * 32, m0, b);
+                        ++n_st;
+                    };
+                    uint32_t ra[32], rb[32];
+                    tmem_ld<32>(t_row, ra);
+                    tmem_ld_wait_tied(ra);
+#pragma unroll 1
+                    for (int c = 0; c < nch; c += 2) {
+                        __syncwarp();
+                        if (c + 1 < nch) tmem_ld<32>(t_row + (c + 1) * 32, rb);
+                        emit(ra, c);
+                        if (c + 1 >= nch) break;
+                        tmem_ld_wait_tied(rb);
+                        __syncwarp();
+                        if (c + 2 < nch) tmem_ld<32>(t_row + (c + 2) * 32, ra);
+                        emit(rb, c + 1);
+                        if (c + 2 < nch) tmem_ld_wait_tied(ra);
+                    }
+                    tc_fence_before();
+                    if (CTAS == 1) mbar_arrive(bar_tempty + 8 * buf);
+                    else           mbar_arrive_cluster(map_to_rank(bar_tempty + 8 * buf, 0));
+                    continue;
+                }
+            }
 #pragma unroll 1
             for (int c = 0; c < ebn / CW; ++c) {
                 const int col0 = n_base + nb * ebn + c * CW;
