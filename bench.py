@@ -586,7 +586,9 @@ def run_ours(args, world, rank, local):
                      "avg_launch_us": round(1e3 * g_ms / n_g, 2)},
         "roofline_quantize": {"bound": "hbm", "achieved": round(quant_gbs, 1), "peak": hbm, "unit": "GB/s",
                               "frac": round(quant_gbs / hbm, 4), "traffic": measured_traffic("quantize"),
-                              "kernel": "quantize_kernel (delayed, 12 launches per step)",
+                              "kernel": "quantize_kernel, delayed, each of the step's 12 tensors in a launch of "
+                                        "its own (the step runs one grouped launch for every W and the first x, "
+                                        "then 7 of these)",
                               "peak_source": f"{peak_src} hbm copy",
                               "algorithmic_bytes_per_launch": round(3 * q_elems / n_q),
                               "avg_launch_us": round(1e3 * q_ms / n_q, 2)},
@@ -871,7 +873,7 @@ def run_configs(fp8, stream, hbm, fp8_peak, reps=20):
     out["nt_256_bias_current"] = {
         "us_quantize_a": round(_time_us(stream, qa, reps), 2), "us_gemm": round(_time_us(stream, mm, reps), 2),
         "us_sequence": round(_time_us(stream, seq, reps), 2), "bound": "latency (0.03 GFLOP, 0.3 MB)",
-        "sequence": "current-scaled quantize of A and of B (each: amax pass + quantize pass), GEMM + bias"}
+        "sequence": "current-scaled quantize of A and of B (one single-block launch each), GEMM + bias"}
 
     # -- square sweep on pre-quantized codes, NT / NN / TN ---------------------
     sq = {}

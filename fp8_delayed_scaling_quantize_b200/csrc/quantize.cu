@@ -283,6 +283,80 @@ quantize_kernel(const void* __restrict__ x, int64_t n, uint8_t* __restrict__ out
     quantize_body<FMT, MODE, IN>(x, n, out8, ring, amax_acc, amax_out, scale_out, blockIdx.x, gridDim.x, s_scale);
 }
 
+// Current scaling of a small tensor in one launch: one block of 1024 threads
+// holds every 8-element unit in registers, reduces the amax, derives the
+// scale and converts, so the call needs neither the accumulator memset nor a
+// second pass over the input (the same arithmetic as the two-pass path, so
+// the same codes, amax and scale). bf16 / fp16 inputs of up to 65536
+// elements.
+constexpr int kSmallThreads = 1024;
+constexpr int kSmallUnits = 8;  // units per thread
+constexpr int64_t kSmallMax = int64_t(kSmallThreads) * kSmallUnits * 8;
+
+template <int FMT, int IN>
+__global__ void __launch_bounds__(kSmallThreads)
+quantize_small_current_kernel(const void* __restrict__ x, int64_t n, uint8_t* __restrict__ out8, float* amax_out,
+                              float* scale_out) {
+    static_assert(IN != FP8_IN_F32, "fp32 units do not fit the registers of a 1024-thread block");
+    __shared__ uint32_t warp_max[kSmallThreads / 32];
+    __shared__ float s_scale;
+    griddep_wait();
+    const int64_t units = n >> 3;
+    const int tail = int(n - (units << 3));
+    Unit v[kSmallUnits];
+#pragma unroll
+    for (int k = 0; k < kSmallUnits; ++k) {
+        const int64_t i = threadIdx.x + int64_t(k) * kSmallThreads;
+        if (i < units) load_unit<IN>(x, i, v[k]);
+    }
+    float t[7];
+    float m = 0.0f;
+    if (threadIdx.x == 0) {
+        for (int j = 0; j < tail; ++j) {
+            t[j] = load_elem<IN>(x, (units << 3) + j);
+            m = fmaxf(m, fabsf(t[j]));
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < kSmallUnits; ++k) {
+        const int64_t i = threadIdx.x + int64_t(k) * kSmallThreads;
+        if (i < units) {
+            float f[8];
+            unit_f32<IN>(v[k], f);
+            amax8(f, m);
+        }
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint32_t bits = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
+    if (lane == 0) warp_max[warp] = bits;
+    __syncthreads();
+    if (warp == 0) {
+        bits = __reduce_max_sync(0xffffffffu, warp_max[lane]);
+        if (lane == 0) {
+            const float a = __uint_as_float(bits);
+            const float sc = (a > 0.0f && isfinite(a)) ? scale_from_amax(fmt_max(FMT), a) : 1.0f;
+            s_scale = sc;
+            *amax_out = a;
+            *scale_out = sc;
+        }
+    }
+    __syncthreads();
+    const float s = s_scale;
+    griddep_launch();
+    uint2* ov = reinterpret_cast<uint2*>(out8);
+#pragma unroll
+    for (int k = 0; k < kSmallUnits; ++k) {
+        const int64_t i = threadIdx.x + int64_t(k) * kSmallThreads;
+        if (i < units) {
+            float f[8], unused = 0.0f;
+            unit_f32<IN>(v[k], f);
+            ov[i] = quant8<FMT>(f, s, unused);
+        }
+    }
+    if (threadIdx.x == 0)
+        for (int j = 0; j < tail; ++j) out8[(units << 3) + j] = uint8_t(cvt_pair<FMT>(__fmul_rn(t[j], s), 0.0f));
+}
+
 // Quantize of a [rows, cols] tensor that also writes the transposed codes
 // [cols, rows] (LAYOUT FP8_QL_COL: only those; FP8_QL_BOTH: both, from one read
 // of the input). A block walks 128 x 64 tiles (rows x columns): each thread
@@ -510,6 +584,13 @@ fp8_status launch_quantize(const void* x, int64_t n, fp8_ring* ring, bool seed, 
     if (ring && !seed)
         return launch_pdl(quantize_kernel<FMT, kDelayed, IN>, grid, kThreads, 0, st, 1, x, n, out8, ring,
                           (uint32_t*)nullptr, amax_out, scale_out);
+    if constexpr (IN != FP8_IN_F32) {
+        // current scaling of a small tensor: one launch (measured on B200, an
+        // NT 256^3 operand: 8.0 us for the memset and two passes)
+        if (!ring && n <= kSmallMax)
+            return launch_pdl(quantize_small_current_kernel<FMT, IN>, 1, kSmallThreads, 0, st, 1, x, n, out8,
+                              amax_out, scale_out);
+    }
     uint32_t* acc = reinterpret_cast<uint32_t*>(amax_out);
     if (cudaMemsetAsync(acc, 0, sizeof(uint32_t), st) != cudaSuccess) return FP8_ERR_CUDA;
     if (launch_pdl(quantize_kernel<FMT, kAmaxOnly, IN>, grid, kThreads, 0, st, 1, x, n, out8, (fp8_ring*)nullptr,

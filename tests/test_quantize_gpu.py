@@ -69,8 +69,10 @@ def test_every_bf16_pattern_under_many_scales(g, fmt):
 
 
 @pytest.mark.parametrize("fmt", [E4M3, E5M2])
-@pytest.mark.parametrize("n", [0, 1, 7, 8, 15, 16, 17, 1000, 4096 * 37 + 5, (1 << 20) + 3])
+@pytest.mark.parametrize("n", [0, 1, 7, 8, 15, 16, 17, 1000, 65535, 65536, 65537, 4096 * 37 + 5, (1 << 20) + 3])
 def test_current_scaling_ragged_sizes(g, fmt, n):
+    """Up to 65536 elements current scaling runs in one single-block launch,
+    above it as an amax pass and a quantize pass: both against the oracle."""
     x = W.bf16_normal((n,), 0.7, 9000 + n)
     q, amax, scale = g.quantize(x.cuda(), fmt, None)
     want, a, s = oracle.quantize_current(x.float().numpy(), fmt)
@@ -268,7 +270,7 @@ def test_f32_inputs_over_the_whole_range(g, fmt):
 
 
 @pytest.mark.parametrize("dtype", [1, 2])
-@pytest.mark.parametrize("n", [1, 7, 9, 1000, 4096 * 37 + 5])
+@pytest.mark.parametrize("n", [1, 7, 9, 1000, 65536, 4096 * 37 + 5])
 def test_f16_f32_ragged_sizes(g, dtype, n):
     import fp8_delayed_scaling_quantize_b200 as fp8
     x = W.bf16_normal((n,), 0.7, 9100 + n).float()
