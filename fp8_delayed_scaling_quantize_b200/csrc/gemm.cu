@@ -79,6 +79,9 @@ struct GemmParams {
     int tma_store;  // tiles leave through shared memory and TMA stores (same conditions)
     // split K: every tile is `split` work units of up to kb_per k-blocks each
     int split, kb_per, total_units;
+    // swapped short problems: the splits of a tile run as one cluster and the
+    // others' fp32 partials reach split 0 through its shared memory (no workspace)
+    int csplit;
     float* ws;         // fp32 partial slots: [tile][rank][split] x (128 x BN)
     uint32_t* ws_cnt;  // per (tile, rank): {units arrived, partials written}
     // FP8 output (fp8_mm_out8): format, delayed-scaling ring, the scale used, the amax
@@ -139,6 +142,18 @@ __device__ __forceinline__ const GroupProblem& group_problem(const GroupTab<true
 
 // Wait for phase `parity` of the mbarrier at `bar`, giving up after
 // `limit_ns`: then the library's device error word is set and false returned.
+__device__ __forceinline__ bool wait_bounded_cluster(uint32_t bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if ((i & 1023u) == 0 && globaltimer_ns() - t0 > limit_ns) {
+            atomicOr(&g_device_error, 1u);
+            return false;
+        }
+    }
+}
+
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
@@ -367,6 +382,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     const uint32_t bar_tempty = bar_tfull + 2 * 8;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBarOffset + (2 * STAGES + 4) * 8);
     uint32_t* ticket_slot = tmem_slot + 1;  // split K: the epilogue's arrival ticket
+    const uint32_t bar_red = smem_addr(tmem_slot + 2);  // cluster split: the other splits' partials are in
     float* s_bias = reinterpret_cast<float*>(smem + L::kBiasOffset);
 
     const int warp = threadIdx.x >> 5;
@@ -386,6 +402,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     const uint32_t idesc = pin(p.idesc);
     int M = pin(p.M), N = pin(p.N);  // per unit in a grouped launch
     int tma_store = pin(p.tma_store), vec_store = pin(p.vec_store);
+    const int csplit = (SWAP && SPLIT) ? pin(p.csplit) : 0;
 
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -396,6 +413,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             mbar_init(bar_tfull + 8 * b, 1);
             mbar_init(bar_tempty + 8 * b, CTAS * kEpiThreads);
         }
+        if (csplit) mbar_init(bar_red, uint32_t(split - 1) * kEpiThreads);
         fence_mbar_init();
         if constexpr (GROUP) {
             for (int i = 0; i < grp.count; ++i) {
@@ -415,7 +433,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     }
     tc_fence_before();
     __syncthreads();
-    if (CTAS == 2) cluster_sync();  // both CTAs' barriers exist before any remote arrive
+    // the cluster's barriers exist before any remote arrive
+    if (CTAS == 2 || csplit) cluster_sync();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     // The prologue above overlaps the previous kernel's tail; operands,
@@ -668,7 +687,34 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             // instruction of a warp covers 512 contiguous bytes.
             constexpr int CW = SWAP ? 16 : 32;  // accumulator columns per TMEM load
             const float4* slots = nullptr;
-            if (SPLIT && split > 1) {
+            if (SPLIT && split > 1 && csplit) {
+                // cluster split: CTA r of the cluster is split r of the tile
+                // (one tile per cluster); splits 1.. push their partials into
+                // split 0's staging area (free in swapped launches), slot r - 1,
+                // laid out as the workspace's slots, and arrive on its barrier
+                if (split_id != 0) {
+                    const uint32_t dst = map_to_rank(stg0 + uint32_t(split_id - 1) * (BM * BN * 4), 0);
+#pragma unroll 1
+                    for (int c = 0; c < BN / CW; ++c) {
+                        if (nb * BN + c * CW >= N) break;  // uniform; split 0 skips it too
+                        uint32_t r[CW];
+                        tmem_ld<CW>(t_row + c * CW, r);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int v = 0; v < CW / 4; ++v)
+                            st_cluster_v4(dst + uint32_t(((c * (CW / 4) + v) * 128 + row_in_tile) * 16),
+                                          __uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                          __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+                    }
+                    mbar_arrive_cluster(map_to_rank(bar_red, 0));  // release: the stores above come first
+                    tc_fence_before();
+                    mbar_arrive(bar_tempty + 8 * buf);
+                    continue;
+                }
+                if (!failed) failed = !wait_bounded_cluster(bar_red, 0);
+                failed = epilogue_bar_or(failed);
+                if (failed) continue;
+            } else if (SPLIT && split > 1) {
                 uint32_t* cnt = p.ws_cnt + 2 * (t * CTAS + int(rank));
                 slots = reinterpret_cast<const float4*>(p.ws) + size_t(t * CTAS + int(rank)) * split * (BM * BN / 4);
                 if (etid == 0) *ticket_slot = atomicAdd(cnt, 1u);
@@ -773,6 +819,20 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
 #pragma unroll
                             for (int i = 0; i < CW; ++i)
                                 acc[i] = sp == 0 ? __uint_as_float(r[i]) : acc[i] + __uint_as_float(r[i]);
+                        } else if (csplit) {
+                            const uint32_t src = stg0 + uint32_t(sp - 1) * (BM * BN * 4) +
+                                                 uint32_t(((c * (CW / 4)) * 128 + row_in_tile) * 16);
+#pragma unroll
+                            for (int v = 0; v < CW / 4; ++v) {
+                                float4 x;
+                                asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                                             : "=f"(x.x), "=f"(x.y), "=f"(x.z), "=f"(x.w)
+                                             : "r"(src + uint32_t(v * 128 * 16)));
+                                acc[4 * v] = acc[4 * v] + x.x;
+                                acc[4 * v + 1] = acc[4 * v + 1] + x.y;
+                                acc[4 * v + 2] = acc[4 * v + 2] + x.z;
+                                acc[4 * v + 3] = acc[4 * v + 3] + x.w;
+                            }
                         } else {
                             const float4* src =
                                 slots + size_t(sp) * (BM * BN / 4) + c * (CW / 4) * 128 + row_in_tile;
@@ -1030,7 +1090,10 @@ fp8_status launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
     p.total_units = int(work);
     const int64_t units_max = sm_count() / CTAS;
     const int units = int(work < units_max ? work : units_max);
-    return launch_pdl(kern, units * CTAS, kThreads, L::kAlloc, st, CTAS, ta, tb, tc, p, GroupTab<false>{});
+    // a cluster split runs each tile's splits as one cluster (every unit in
+    // the grid's one round, so the grid is a whole number of clusters)
+    const int cluster = p.csplit ? p.split : CTAS;
+    return launch_pdl(kern, units * CTAS, kThreads, L::kAlloc, st, cluster, ta, tb, tc, p, GroupTab<false>{});
 }
 
 template <int BN, bool A_MN, bool B_MN, int STAGES, int CTAS, bool SWAP = false, bool OUT8 = false>
@@ -1184,17 +1247,28 @@ fp8_status dispatch_swap(const uint8_t* a8, int fa, const uint8_t* b8, int fb, i
                          int64_t batch, int64_t stride_a, int64_t stride_b, GemmParams p, void* ws, size_t ws_bytes,
                          int split_req, cudaStream_t st) {
     const int bn = swap_bn(M);
-    // the automatic choice splits only with a workspace to split into
-    p.split = swap_split(M, N, K, batch, split_req == 0 && !ws ? 1 : split_req, sm_count());
+    // The automatic choice without a workspace splits as a cluster: the
+    // splits' partials go through split 0's staging area, which holds three
+    // 128 x 16 partials or one 128 x 32 one.
+    p.csplit = 0;
+    if (split_req == 0 && !ws) {
+        const int s_max = bn == 16 ? 4 : 2;
+        int s = swap_split(M, N, K, batch, 0, sm_count());
+        s = s > s_max ? s_max : s;
+        p.split = s;
+        p.csplit = s > 1;
+    } else {
+        p.split = swap_split(M, N, K, batch, split_req, sm_count());
+    }
     if (p.split == 0) return FP8_ERR_UNSUPPORTED;
-    if (p.split > 1) {
+    if (p.split > 1 && !p.csplit) {
         const int64_t tiles = ((N + BM - 1) / BM) * batch;
         if (!ws || ws_bytes < split_ws_bytes(tiles, 1, bn, p.split)) {
             if (split_req >= 2) return FP8_ERR_INVALID_ARG;
             p.split = 1;  // an automatic split that does not fit the workspace is dropped
         }
     }
-    if (p.split > 1) {
+    if (p.split > 1 && !p.csplit) {
         p.ws_cnt = static_cast<uint32_t*>(ws);
         p.ws = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kSplitCntBytes);
     }

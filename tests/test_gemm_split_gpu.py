@@ -165,8 +165,8 @@ def test_one_workspace_serves_a_sequence_and_graph_replay(g):
 def test_automatic_split_of_short_problems(g, layout, M, N, K):
     """split_k = 0 with a workspace: short problems with a long K split on
     their own (the workspace size query says how much they need); the result
-    is the oracle's, bit-identical run to run, and fp8_mm (no workspace, no
-    split) agrees within the same bar."""
+    is the oracle's, bit-identical run to run, and fp8_mm (no workspace)
+    gives the same bits."""
     import fp8_delayed_scaling_quantize_b200 as fp8
     need = fp8.fp8_mm_workspace_size(M, N, K, 1, layout, 0)
     assert need > 4096, "the automatic choice is expected to split this shape"
@@ -179,5 +179,28 @@ def test_automatic_split_of_short_problems(g, layout, M, N, K):
     y, s = _oracle(c, layout, M, N, K, E4M3, E4M3, 1)
     tol = oracle.tolerance(y, s)
     g.assert_within(out.float().cpu().numpy().reshape(y.shape), y, tol, f"auto split {M}x{N}x{K}")
+    # fp8_mm (no workspace) splits the same way as a cluster, the other splits'
+    # partials reaching split 0 through its shared memory: the same sum in the
+    # same order, so the same bits
     plain = _run(g, c, layout, M, N, K, E4M3, E4M3, 1, None, 0)
-    g.assert_within(plain.float().cpu().numpy().reshape(y.shape), y, tol, f"no split {M}x{N}x{K}")
+    assert torch.equal(plain.view(torch.int16), out.view(torch.int16))
+
+
+# Cluster splits of short problems (fp8_mm, no workspace): ragged N, bias,
+# batches with B broadcast; 16-row tiles split up to 4 ways, 32-row tiles 2
+# ways. Against the oracle in full and the workspace split with the same
+# number of splits bit for bit.
+@pytest.mark.parametrize("layout,M,N,K,batch,bias_kind,split", [
+    (NT, 5, 1000, 4096, 2, 1, 4), (NN, 12, 2048, 3072, 1, 2, 4), (NT, 24, 2048, 4096, 1, 1, 2),
+    (NN, 32, 1024, 8192, 1, 0, 2)])
+def test_cluster_split_of_short_problems(g, layout, M, N, K, batch, bias_kind, split):
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    c = _case(layout, M, N, K, E4M3, E5M2, 1800 + M + N, batch=batch, bcast_b=batch > 1, bias_kind=bias_kind)
+    plain = _run(g, c, layout, M, N, K, E4M3, E5M2, batch, None, 0)
+    ws = g.workspace(fp8.fp8_mm_workspace_size(M, N, K, batch, layout, split))
+    forced = _run(g, c, layout, M, N, K, E4M3, E5M2, batch, ws, split)
+    assert torch.equal(plain.view(torch.int16), forced.view(torch.int16))
+    y, s = _oracle(c, layout, M, N, K, E4M3, E5M2, batch)
+    g.assert_within(plain.float().cpu().numpy().reshape(y.shape), y, oracle.tolerance(y, s),
+                    f"cluster split {M}x{N}x{K}")
+    assert fp8.fp8_last_device_error() == fp8.FP8_OK
