@@ -230,7 +230,11 @@ FP8LITE_API fp8_status fp8_quantize_many_ex(const fp8_quantize_job* jobs, int32_
  *   out[b,i,j] = bf16_rne( (sum_k op(A_b)[i,k] op(B_b)[k,j]) / (sa*sb) + bias_j )
  *
  * accumulated in fp32 on the tensor cores, the scale and the bias applied in
- * fp32, then ONE rounding to bf16. bias_j is bias[j] (bf16) when bias_scale
+ * fp32, then ONE rounding to bf16. Short problems (M <= 32 in NT or NN) with a
+ * long K may be split along K as a cluster of 2 .. 4 CTAs that add their
+ * fp32 partials in split order through shared memory (no workspace); the
+ * result is then what fp8_mm_ws gives with that split, and it does not
+ * depend on timing. bias_j is bias[j] (bf16) when bias_scale
  * is NULL, dec(bias[j]) / *bias_scale (fp8 codes of bias_fmt) when it is not,
  * 0 when bias is NULL; the bias is broadcast over rows and batches.
  *
@@ -279,7 +283,9 @@ FP8LITE_API fp8_status fp8_mm(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8, 
  *                 partials' round trip through L2 cost more than the shorter
  *                 main loop saved);
  *                 1: no split; 2 .. 4: exactly that many splits.
- * workspace       NULL (no split), else device memory,
+ * workspace       NULL: as fp8_mm (split_k 0: a short problem may split as a
+ *                 cluster, without a workspace; 1: no split; 2 .. 4 need a
+ *                 workspace), else device memory,
  *                 16-byte aligned, of workspace_bytes >=
  *                 fp8_mm_workspace_size(..., split_k) bytes. Its first 4096
  *                 bytes are counters: they must be zero before the first call
