@@ -504,3 +504,41 @@ def test_exchange_helper_on_one_rank(g):
             assert np.array_equal(hist, refs[i].hist) and rs == refs[i].scale and acc == 0
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("fmt", [E4M3, E5M2])
+def test_more_than_2_to_31_elements(g, fmt):
+    """A tensor past 2^31 elements (4 GB of bf16, with a ragged tail): every
+    bf16 bit pattern repeated, quantized with a delayed scale. The codes at
+    sampled positions (including the last 1 M and the tail) equal the
+    oracle's codes of the same pattern, the amax is +inf (the infinite
+    patterns; NaN is ignored) and the ring keeps its scale, as the oracle's
+    ring does."""
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    n = (1 << 31) + 19
+    pats = W.bf16_bit_patterns()
+    x = pats.cuda().repeat(n // 65536 + 1)[:n].contiguous()
+    s = np.float32(2.0 ** -4)
+    ring = g.new_ring()
+    host = fp8.fp8_ring()
+    host.scale = float(s)
+    fp8.fp8_ring_set(ring, host)
+    q = torch.empty(n, dtype=torch.uint8, device="cuda")
+    amax = torch.empty(1, device="cuda")
+    sc = torch.empty(1, device="cuda")
+    fp8.fp8_quantize(x, n, fmt, ring, q, amax, sc)
+    want = oracle.quantize_with_scale(pats.float().numpy(), s, fmt)
+    rng = np.random.default_rng(7 + fmt)
+    idx = np.concatenate([rng.integers(0, n, 200000), np.arange(n - (1 << 20), n)])
+    got = q[torch.from_numpy(idx).cuda()].cpu().numpy()
+    ref = want[idx % 65536]
+    nan = _nan_code(ref, fmt)
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert _nan_code(got[nan], fmt).all()
+    assert g.f32(sc)[0] == s and g.f32(amax)[0] == np.inf
+    r = oracle.DelayedRing(float(s))
+    r.fold(np.float32(np.inf), fmt)
+    hist, rs, idx_, acc, ticket = g.ring_state(ring)
+    assert np.array_equal(hist, r.hist) and rs == r.scale and idx_ == r.idx and acc == 0 and ticket == 0
+    del x, q
+    torch.cuda.empty_cache()
