@@ -204,3 +204,31 @@ def test_cluster_split_of_short_problems(g, layout, M, N, K, batch, bias_kind, s
     g.assert_within(plain.float().cpu().numpy().reshape(y.shape), y, oracle.tolerance(y, s),
                     f"cluster split {M}x{N}x{K}")
     assert fp8.fp8_last_device_error() == fp8.FP8_OK
+
+
+def test_cluster_split_in_a_cuda_graph(g):
+    """A short problem that splits as a cluster, captured in a CUDA graph and
+    replayed on new operands: every replay equals a fresh eager call."""
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    M, N, K = 8, 2048, 4096
+    c = _case(NT, M, N, K, E4M3, E4M3, 1900)
+    a, b = c["a8"].cuda(), c["b8"].cuda()
+    sa = torch.tensor([0.75], device="cuda")
+    sb = torch.tensor([1.5], device="cuda")
+    out = torch.empty(M * N, dtype=torch.bfloat16, device="cuda")
+    st = torch.cuda.Stream()
+    st.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(st):
+        g.mm(a, E4M3, b, E4M3, sa, sb, NT, M, N, K, out=out)
+    torch.cuda.current_stream().wait_stream(st)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        g.mm(a, E4M3, b, E4M3, sa, sb, NT, M, N, K, out=out)
+    for seed in (1901, 1902, 1903):
+        a.copy_(W.fp8_codes((M * K,), E4M3, seed).cuda())
+        graph.replay()
+        want = _run(g, dict(c, a8=a.cpu()), NT, M, N, K, E4M3, E4M3, 1, None, 0)
+        torch.cuda.synchronize()
+        assert torch.equal(out.view(torch.int16), want.view(torch.int16))
+    del graph
+    assert fp8.fp8_last_device_error() == fp8.FP8_OK
