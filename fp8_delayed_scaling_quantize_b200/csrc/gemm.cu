@@ -11,8 +11,10 @@
 // Design (B200-first; the pages' sm_89 mma.sync / ldmatrix / cp.async / PRMT
 // kernel is prior art only):
 //  * persistent CTAs (one per SM at most), each walking output tiles
-//    BM x BN = 128 x {64,128,256} in M-fastest order so CTAs that run together
-//    share the B (weight) tile in L2;
+//    BM x BN = 128 x {64,128,256}, or 256 x 256 on an SM pair (tcgen05
+//    cta_group::2, clusters of two, no TMA multicast), in groups of M-tile
+//    rows walked M-fastest, so that the tiles running together share their
+//    A and B panels in L2;
 //  * 6 warps with fixed roles: warp 0 issues TMA loads (one lane), warp 1
 //    owns TMEM and issues tcgen05.mma (one lane), warps 2-5 run the epilogue
 //    (one per TMEM lane quarter);
@@ -29,9 +31,15 @@
 //    bias in fp32 (one fma), one round-to-nearest-even to bf16, staged as
 //    128 x 32 tiles in shared memory and written by one TMA store each (TMA
 //    clips the M / N tails);
-//  * split K (with a caller workspace): a tile's k-blocks are shared by
-//    several CTAs; the last to finish adds the others' fp32 partials in split
-//    order and runs the epilogue;
+//  * short problems (M <= 32, NT and NN) swap the operands, C^T = B^T A^T,
+//    so that C's few rows become an MMA N of 16 or 32;
+//  * split K: a tile's k-blocks are shared by several CTAs, whose fp32
+//    partials go through a caller workspace (the last CTA to finish adds
+//    them), through the library's static scratch, or, for short problems
+//    without a workspace, to split 0 of a cluster through distributed shared
+//    memory; partials are always added in split order;
+//  * grouped launches: up to 4 problems (a linear's dX and dW) share one
+//    persistent grid, each work unit looking up its problem in a table;
 //  * every mbarrier wait is bounded by a time limit; a wait that gives up
 //    records FP8_ERR_DEVICE_TIMEOUT in the library's device error word and the
 //    CTA stops issuing work and exits through the normal teardown.
@@ -1116,21 +1124,23 @@ fp8_status launch(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, co
 // Tile choice for 148 SMs by a small cost model: a persistent grid walks
 // ceil(units / CTAs) rounds of work units, each costing its k-blocks times
 // the per-k-block time of that tile shape, plus the one epilogue left exposed
-// at the end. The per-k-block times (microseconds at the clocks seen under
-// load) and epilogue times were measured on B200 with this kernel: 128x256
-// 0.48, 128x128 0.40, 128x64 0.30, an SM pair's 256x256 0.43 and 256x128
-// 0.25. An SM pair's 256 x 128 tile loads 24 KB per SM per k-block, so eight
-// stages keep its MMAs fed; a single SM's 128 x 128 tile needs 32 KB per
-// k-block for half the MMA work and waits on its loads. Pairs of 256 x 256
-// are used only with at least one such tile per SM (below that their coarser
-// grain loses). MN-major B needs whole 128-byte swizzle atoms along N per
-// CTA, so the 256 x 128 pair tile takes K-major B only.
+// at the end. The per-k-block and epilogue constants were fitted on B200 to
+// this kernel: 128x256 0.48, 128x128 0.40, 128x64 0.30 and an SM pair's
+// 256x256 0.43. While its tensor core runs, an SM takes in operands at about
+// 65 bytes per clock, so a one-SM k-block costs more than its MMAs (a
+// 128 x 128 k-block loads 32 KB for half the MMA work of a 128 x 256 one,
+// which loads 48 KB), and the wider tile costs less per output. Pairs of
+// 256 x 256 are used only with at least one such tile per SM (below that
+// their coarser grain loses). The pair's 256 x 128 tile (24 KB per SM per
+// k-block) measured slower than one SM's 128 x 128 on the shapes it could
+// serve and is not chosen.
 //
 // Split K (split_req >= 2, with a workspace): a tile becomes `split` units
 // over consecutive k-block ranges; the unit that finishes last adds the
 // others' fp32 partials and runs the epilogue. The automatic choice
-// (split_req = 0) does not split: on every shape measured on B200 the
-// partials' round trip through L2 cost more than the shorter main loop saved.
+// (split_req = 0) does not split these unswapped tiles: on every shape
+// measured on B200 the partials' round trip through L2 cost more than the
+// shorter main loop saved (short problems, swapped below, do split).
 constexpr size_t kSplitCntBytes = 4096;  // two counters per (tile, CTA of the tile)
 constexpr int kMaxSplit = 4;
 
