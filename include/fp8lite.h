@@ -111,7 +111,9 @@ FP8LITE_API fp8_status fp8_ring_set(fp8_ring* ring, const fp8_ring* host, void* 
  *   accumulators [fp8.py@4dc5e923, bullet on the last-block epilogue].
  * ring == NULL -- current ("dynamic") scaling [fp8.py@4dc5e923, bullet on
  *   the dynamic path]: s = fmt_max / amax(x) (1 if amax is 0 or not finite);
- *   a memset and two launches (amax pass, quantize pass).
+ *   one launch for bf16/fp16 tensors of up to 65536 elements (one thread
+ *   block holds the whole tensor), otherwise a memset and two launches (amax
+ *   pass, quantize pass).
  * fmt_max / m is an IEEE fp32 division; an overflow is clamped to FLT_MAX.
  *
  * x          device, bf16[n], 16-byte aligned
