@@ -44,6 +44,11 @@ def bf16_normal(shape, std: float, seed: int) -> torch.Tensor:
     return (x * std).to(torch.bfloat16)
 
 
+def f32_normal(shape, std: float, seed: int) -> torch.Tensor:
+    """fp32 tensor ~ N(0, std^2) on the CPU."""
+    return torch.randn(tuple(shape), generator=_gen(seed), dtype=torch.float32) * std
+
+
 def uniform(lo: float, hi: float, seed: int, n: int = 1) -> torch.Tensor:
     """fp32 tensor of n draws ~ U(lo, hi)."""
     u = torch.rand(n, generator=_gen(seed), dtype=torch.float32)
