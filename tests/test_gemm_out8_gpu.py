@@ -127,3 +127,24 @@ def test_out8_feeds_the_next_gemm(g):
     y2 = g.mm(out, E4M3, w2.cuda(), E4M3, sc, one, NT, M, N2, N)
     want, s = oracle.mm(out.cpu().numpy(), E4M3, w2.numpy(), E4M3, float(g.f32(sc)[0]), 1.0, NT, M, N2, N)
     g.assert_within(y2.float().cpu().numpy().reshape(M, N2), want[0], oracle.tolerance(want[0], s[0]), "chain")
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_out8_random_problems(g, seed):
+    """Drawn problems (layout, formats, output format, sizes with the pitch
+    rules kept and at least 4096 outputs, batches with B broadcast, padding,
+    bias kind), each over three ring steps."""
+    rng = np.random.default_rng(47000 + seed)
+    layout = int(rng.choice([NT, NN, TN]))
+    fa, fb, out_fmt = (int(v) for v in rng.integers(0, 2, 3))
+    M = int(rng.integers(1, 40)) * 16 if layout == TN else int(rng.integers(16, 640))
+    N = int(rng.integers(4, 40)) * 16 if layout != NT else int(rng.integers(64, 640))
+    N = max(N, (4096 + M - 1) // M if layout == NT else N)
+    K = int(rng.integers(1, 48)) * 16 if layout != TN else int(rng.integers(1, 768))
+    batch = int(rng.choice([1, 1, 2]))
+    bcast_b = batch > 1 and rng.random() < 0.5
+    pad_c = int(rng.choice([0, 5, 16])) if batch > 1 else 0
+    if M * N < 4096:
+        M = (4096 + N - 1) // N if layout != TN else ((4096 + N - 1) // N + 15) // 16 * 16
+    _run_case(g, layout, M, N, K, fa, fb, out_fmt, 48000 + 10 * seed, batch=batch, bcast_b=bcast_b,
+              bias_kind=int(rng.integers(0, 3)), pad_c=pad_c)

@@ -96,3 +96,80 @@ def test_random_call_sequence(g, seed):
         assert np.array_equal(hist, ref.hist) and rs == ref.scale and idx == ref.idx, what
         assert acc == 0 and ticket == 0, what
     assert fp8.fp8_last_device_error() == fp8.FP8_OK
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_random_grouped_jobs(g, seed):
+    """fp8_quantize_many with 1 .. 8 drawn jobs (own ring, format, input type
+    and size each), three calls in a row: every job equals the oracle's
+    delayed call on its own ring, bit for bit."""
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    rng = np.random.default_rng(43000 + seed)
+    count = int(rng.integers(1, 9))
+    fmts = [int(v) for v in rng.integers(0, 2, count)]
+    rings = [g.new_ring() for _ in range(count)]
+    refs = [oracle.DelayedRing() for _ in range(count)]
+    for call in range(3):
+        drawn = [_input(rng, 44000 + 100 * seed + 10 * call + j) for j in range(count)]
+        outs = [torch.empty(max(x.numel(), 1), dtype=torch.uint8, device="cuda") for _, x in drawn]
+        amaxs = [torch.full((1,), -1.0, device="cuda") for _ in range(count)]
+        scales = [torch.full((1,), -1.0, device="cuda") for _ in range(count)]
+        xd = [x.cuda() if x.numel() else None for _, x in drawn]
+        fp8.fp8_quantize_many([(xd[j], drawn[j][1].numel(), fmts[j], rings[j], outs[j] if xd[j] is not None else None,
+                                amaxs[j], scales[j], drawn[j][0]) for j in range(count)])
+        for j, (dtype, x) in enumerate(drawn):
+            what = f"call {call} job {j} dtype {dtype} n {x.numel()} fmt {fmts[j]}"
+            xf = x.float().numpy()
+            s = np.float32(refs[j].scale)
+            a = oracle.amax(xf)
+            refs[j].fold(a, fmts[j])
+            assert np.array_equal(g.codes(outs[j])[:x.numel()], _oracle_codes(x, s, fmts[j])), what
+            assert g.f32(scales[j])[0] == s and g.f32(amaxs[j])[0] == np.float32(a), what
+            hist, rs, idx, acc, ticket = g.ring_state(rings[j])
+            assert np.array_equal(hist, refs[j].hist) and rs == refs[j].scale and idx == refs[j].idx, what
+            assert acc == 0 and ticket == 0, what
+    assert fp8.fp8_last_device_error() == fp8.FP8_OK
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_random_dual_quantize(g, seed):
+    """fp8_quantize_2d on drawn shapes (multiples of 8), input types and
+    layouts, delayed or current: the row-major codes are the oracle's and
+    the transposed copy holds the same bytes."""
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    rng = np.random.default_rng(45000 + seed)
+    fmt = int(rng.integers(0, 2))
+    ring = g.new_ring() if rng.random() < 0.7 else None
+    ref = oracle.DelayedRing()
+    for call in range(3):
+        rows, cols = (int(v) * 8 for v in rng.integers(1, 160, 2))
+        dtype = int(rng.choice([0, 1, 2]))
+        sigma = float(10 ** rng.uniform(-3, 2))
+        seed_x = 46000 + 10 * seed + call
+        x = (W.bf16_normal((rows, cols), sigma, seed_x) if dtype == 0
+             else W.f32_normal((rows, cols), sigma, seed_x).to(DTYPES[dtype]))
+        layout = int(rng.choice([fp8.FP8_QL_COL, fp8.FP8_QL_BOTH]))
+        out = torch.full((rows * cols,), 0xAB, dtype=torch.uint8, device="cuda")
+        out_t = torch.full((rows * cols,), 0xCD, dtype=torch.uint8, device="cuda")
+        amax = torch.full((1,), -1.0, device="cuda")
+        scale = torch.full((1,), -1.0, device="cuda")
+        fp8.fp8_quantize_2d(x.cuda(), dtype, rows, cols, fmt, ring, 0, layout, out, out_t, amax, scale)
+        xf = x.float().numpy().reshape(-1)
+        a = oracle.amax(xf)
+        if ring is None:
+            s = oracle.current_scale(a, fmt)
+        else:
+            s = np.float32(ref.scale)
+            ref.fold(a, fmt)
+        want = _oracle_codes(x.reshape(-1), s, fmt)
+        what = f"call {call} {rows}x{cols} dtype {dtype} layout {layout}"
+        assert np.array_equal(g.codes(out_t).reshape(cols, rows), want.reshape(rows, cols).T), what
+        if layout == fp8.FP8_QL_BOTH:
+            assert np.array_equal(g.codes(out), want), what
+        else:
+            assert (g.codes(out) == 0xAB).all(), what
+        assert g.f32(scale)[0] == np.float32(s) and g.f32(amax)[0] == np.float32(a), what
+        if ring is not None:
+            hist, rs, idx, acc, ticket = g.ring_state(ring)
+            assert np.array_equal(hist, ref.hist) and rs == ref.scale and idx == ref.idx, what
+            assert acc == 0 and ticket == 0, what
