@@ -1162,9 +1162,11 @@ def run_kernel(args):
         for i in range(max(args.warmup, 3)):
             call(i)
     torch.cuda.synchronize()
-    hold_stream(st)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(torch.cuda.current_device()) as clocks:
+        # the hold starts after the sampler's set-up, so it still covers the
+        # host's enqueueing of every timed launch
+        hold_stream(st, 2000 + 40 * reps)
         with torch.cuda.stream(st):
             e0.record(st)
             for i in range(reps):
