@@ -866,14 +866,25 @@ def run_configs(fp8, stream, hbm, fp8_peak, reps=20):
     qb = lambda i: fp8.fp8_quantize(b, N * K, E4M3, None, b8, bm, sb, stream=stream)
     mm = lambda i: fp8.fp8_mm(a8, E4M3, b8, E4M3, sa, sb, NT, M, N, K, 1, 0, 0, 0, bias, None, 0, y, stream=stream)
 
+    qab = lambda i: fp8.fp8_quantize_current_many([(a, M * K, E4M3, None, a8, am, sa), (b, N * K, E4M3, None, b8, bm, sb)],
+                                                  stream=stream)
+
     def seq(i):
         qa(i)
         qb(i)
         mm(i)
+
+    def seq_grouped(i):
+        qab(i)
+        mm(i)
     out["nt_256_bias_current"] = {
         "us_quantize_a": round(_time_us(stream, qa, reps), 2), "us_gemm": round(_time_us(stream, mm, reps), 2),
-        "us_sequence": round(_time_us(stream, seq, reps), 2), "bound": "latency (0.03 GFLOP, 0.3 MB)",
-        "sequence": "current-scaled quantize of A and of B (one single-block launch each), GEMM + bias"}
+        "us_sequence": round(_time_us(stream, seq, reps), 2),
+        "us_quantize_a_and_b_one_launch": round(_time_us(stream, qab, reps), 2),
+        "us_sequence_grouped": round(_time_us(stream, seq_grouped, reps), 2),
+        "bound": "latency (0.03 GFLOP, 0.3 MB)",
+        "sequence": "current-scaled quantize of A and of B (one single-block launch each), GEMM + bias; "
+                    "grouped: A and B current-scaled in one launch (fp8_quantize_current_many), GEMM + bias"}
 
     # -- square sweep on pre-quantized codes, NT / NN / TN ---------------------
     sq = {}

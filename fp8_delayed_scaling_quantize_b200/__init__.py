@@ -46,6 +46,7 @@ class fp8_ring(ctypes.Structure):
 assert ctypes.sizeof(fp8_ring) == FP8_RING_BYTES
 
 FP8_QUANTIZE_MAX_JOBS = 8
+FP8_QUANTIZE_SMALL_MAX = 65536
 
 
 class fp8_quantize_job(ctypes.Structure):
@@ -91,6 +92,7 @@ def _load():
         "fp8_bias_grad": (I, [P, I64, I64, P, P]),
         "fp8_quantize_many": (I, [P, ctypes.c_int32, P]),
         "fp8_quantize_many_ex": (I, [P, ctypes.c_int32, ctypes.c_uint32, P]),
+        "fp8_quantize_current_many": (I, [P, ctypes.c_int32, P]),
         "fp8_rings_fold": (I, [P, ctypes.c_int32, P, P]),
         "fp8_mm_ws": (I, [P, I, P, I, P, P, I, I64, I64, I64, I64, I64, I64, I64, P, P, I, P, P, ctypes.c_size_t,
                           ctypes.c_int32, P]),
@@ -183,15 +185,26 @@ def fp8_rings_fold(rings, count, fmts, stream=None):
                   "fp8_rings_fold")
 
 
-def fp8_quantize_many(jobs, stream=None, flags=0):
-    """jobs: sequence of (x, n, fmt, ring, out8, amax_out, scale_out[, dtype])."""
+def _jobs(jobs):
     arr = (fp8_quantize_job * max(len(jobs), 1))()
     for i, job in enumerate(jobs):
         x, n, fmt, ring, out8, amax_out, scale_out = job[:7]
         dtype = job[7] if len(job) > 7 else FP8_IN_BF16
         arr[i] = fp8_quantize_job(_ptr(x), int(n), int(fmt), int(dtype), _ptr(ring), _ptr(out8), _ptr(amax_out),
                                   _ptr(scale_out))
-    return _check(lib.fp8_quantize_many_ex(ctypes.cast(arr, ctypes.c_void_p), len(jobs), int(flags),
+    return arr
+
+
+def fp8_quantize_current_many(jobs, stream=None):
+    """jobs: sequence of (x, n, fmt, None, out8, amax_out, scale_out[, dtype]),
+    each current-scaled; bf16/fp16 of at most FP8_QUANTIZE_SMALL_MAX elements."""
+    return _check(lib.fp8_quantize_current_many(ctypes.cast(_jobs(jobs), ctypes.c_void_p), len(jobs),
+                                                _stream(stream)), "fp8_quantize_current_many")
+
+
+def fp8_quantize_many(jobs, stream=None, flags=0):
+    """jobs: sequence of (x, n, fmt, ring, out8, amax_out, scale_out[, dtype])."""
+    return _check(lib.fp8_quantize_many_ex(ctypes.cast(_jobs(jobs), ctypes.c_void_p), len(jobs), int(flags),
                                            _stream(stream)), "fp8_quantize_many")
 
 

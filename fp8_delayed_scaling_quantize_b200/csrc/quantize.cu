@@ -294,13 +294,10 @@ constexpr int kSmallUnits = 8;  // units per thread
 constexpr int64_t kSmallMax = int64_t(kSmallThreads) * kSmallUnits * 8;
 
 template <int FMT, int IN>
-__global__ void __launch_bounds__(kSmallThreads)
-quantize_small_current_kernel(const void* __restrict__ x, int64_t n, uint8_t* __restrict__ out8, float* amax_out,
-                              float* scale_out) {
+__device__ __forceinline__ void small_current_body(const void* __restrict__ x, int64_t n, uint8_t* __restrict__ out8,
+                                                   float* amax_out, float* scale_out, uint32_t (&warp_max)[32],
+                                                   float& s_scale) {
     static_assert(IN != FP8_IN_F32, "fp32 units do not fit the registers of a 1024-thread block");
-    __shared__ uint32_t warp_max[kSmallThreads / 32];
-    __shared__ float s_scale;
-    griddep_wait();
     const int64_t units = n >> 3;
     const int tail = int(n - (units << 3));
     Unit v[kSmallUnits];
@@ -336,7 +333,7 @@ quantize_small_current_kernel(const void* __restrict__ x, int64_t n, uint8_t* __
             const float a = __uint_as_float(bits);
             const float sc = (a > 0.0f && isfinite(a)) ? scale_from_amax(fmt_max(FMT), a) : 1.0f;
             s_scale = sc;
-            *amax_out = a;
+            if (amax_out) *amax_out = a;
             *scale_out = sc;
         }
     }
@@ -355,6 +352,53 @@ quantize_small_current_kernel(const void* __restrict__ x, int64_t n, uint8_t* __
     }
     if (threadIdx.x == 0)
         for (int j = 0; j < tail; ++j) out8[(units << 3) + j] = uint8_t(cvt_pair<FMT>(__fmul_rn(t[j], s), 0.0f));
+}
+
+template <int FMT, int IN>
+__global__ void __launch_bounds__(kSmallThreads)
+quantize_small_current_kernel(const void* __restrict__ x, int64_t n, uint8_t* __restrict__ out8, float* amax_out,
+                              float* scale_out) {
+    __shared__ uint32_t warp_max[kSmallThreads / 32];
+    __shared__ float s_scale;
+    griddep_wait();
+    small_current_body<FMT, IN>(x, n, out8, amax_out, scale_out, warp_max, s_scale);
+}
+
+// Current scaling of up to FP8_QUANTIZE_MAX_JOBS small tensors in one
+// launch: block j runs job j exactly as quantize_small_current_kernel runs a
+// single tensor (so the same codes, amax and scale).
+struct SmallJobs {
+    const void* x[FP8_QUANTIZE_MAX_JOBS];
+    int64_t n[FP8_QUANTIZE_MAX_JOBS];
+    uint8_t* out8[FP8_QUANTIZE_MAX_JOBS];
+    float* amax_out[FP8_QUANTIZE_MAX_JOBS];
+    float* scale_out[FP8_QUANTIZE_MAX_JOBS];
+    int kind[FP8_QUANTIZE_MAX_JOBS];  // 2 * fmt + dtype (bf16 or fp16)
+};
+
+__global__ void __launch_bounds__(kSmallThreads) quantize_small_current_many_kernel(const __grid_constant__ SmallJobs q) {
+    __shared__ uint32_t warp_max[kSmallThreads / 32];
+    __shared__ float s_scale;
+    griddep_wait();
+    const int j = blockIdx.x;
+    switch (q.kind[j]) {
+        case 2 * FP8_E4M3 + FP8_IN_BF16:
+            small_current_body<FP8_E4M3, FP8_IN_BF16>(q.x[j], q.n[j], q.out8[j], q.amax_out[j], q.scale_out[j],
+                                                      warp_max, s_scale);
+            break;
+        case 2 * FP8_E4M3 + FP8_IN_F16:
+            small_current_body<FP8_E4M3, FP8_IN_F16>(q.x[j], q.n[j], q.out8[j], q.amax_out[j], q.scale_out[j],
+                                                     warp_max, s_scale);
+            break;
+        case 2 * FP8_E5M2 + FP8_IN_BF16:
+            small_current_body<FP8_E5M2, FP8_IN_BF16>(q.x[j], q.n[j], q.out8[j], q.amax_out[j], q.scale_out[j],
+                                                      warp_max, s_scale);
+            break;
+        default:
+            small_current_body<FP8_E5M2, FP8_IN_F16>(q.x[j], q.n[j], q.out8[j], q.amax_out[j], q.scale_out[j],
+                                                     warp_max, s_scale);
+            break;
+    }
 }
 
 // Quantize of a [rows, cols] tensor that also writes the transposed codes
@@ -816,4 +860,25 @@ extern "C" fp8_status fp8_quantize_many_ex(const fp8_quantize_job* jobs, int32_t
 
 extern "C" fp8_status fp8_quantize_many(const fp8_quantize_job* jobs, int32_t count, void* stream) {
     return fp8_quantize_many_ex(jobs, count, 0u, stream);
+}
+
+extern "C" fp8_status fp8_quantize_current_many(const fp8_quantize_job* jobs, int32_t count, void* stream) {
+    if (!jobs || count < 1 || count > FP8_QUANTIZE_MAX_JOBS) return FP8_ERR_INVALID_ARG;
+    SmallJobs q = {};
+    for (int j = 0; j < count; ++j) {
+        const fp8_quantize_job& in = jobs[j];
+        if (!valid_fmt(in.fmt) || !valid_dtype(in.dtype)) return FP8_ERR_INVALID_ARG;
+        if (in.ring || !in.scale_out || in.n < 0) return FP8_ERR_INVALID_ARG;
+        if (in.n > 0 && (!in.x || !in.out8)) return FP8_ERR_INVALID_ARG;
+        if (in.dtype == FP8_IN_F32 || in.n > kSmallMax) return FP8_ERR_UNSUPPORTED;
+        if (!aligned(in.x, 16) || !aligned(in.out8, 16)) return FP8_ERR_ALIGNMENT;
+        if (!aligned(in.scale_out, 4) || !aligned(in.amax_out, 4)) return FP8_ERR_ALIGNMENT;
+        q.x[j] = in.x;
+        q.n[j] = in.n;
+        q.out8[j] = in.out8;
+        q.amax_out[j] = in.amax_out;
+        q.scale_out[j] = in.scale_out;
+        q.kind[j] = 2 * int(in.fmt) + int(in.dtype);
+    }
+    return launch_pdl(quantize_small_current_many_kernel, count, kSmallThreads, 0, as_stream(stream), 1, q);
 }

@@ -26,7 +26,7 @@
 extern "C" {
 #endif
 
-#define FP8LITE_ABI_VERSION 3
+#define FP8LITE_ABI_VERSION 4
 
 /* Exported entry points (the library is built with hidden visibility). */
 #if defined(__GNUC__)
@@ -224,6 +224,20 @@ FP8LITE_API fp8_status fp8_quantize_many(const fp8_quantize_job* jobs, int32_t c
  * all-reduce and fp8_rings_fold; see fp8_quantize_ex). */
 FP8LITE_API fp8_status fp8_quantize_many_ex(const fp8_quantize_job* jobs, int32_t count, uint32_t flags,
                                             void* stream);
+
+/* Current ("dynamic") scaling of up to FP8_QUANTIZE_MAX_JOBS small tensors in
+ * ONE launch, e.g. the two operands of a small GEMM [fp8.py@4dc5e923, bullet
+ * on the dynamic path]. Each job is exactly an fp8_quantize_ex call with
+ * ring == NULL: s = fmt_max / amax(x) (1 if amax is 0 or not finite), the
+ * same codes, amax and scale. One thread block per job holds the whole
+ * tensor, so every job must be bf16 or fp16 (dtype) with
+ * 0 <= n <= FP8_QUANTIZE_SMALL_MAX elements; ring must be NULL; amax_out is
+ * optional, scale_out required; x and out8 16-byte aligned.
+ * Errors: FP8_ERR_INVALID_ARG (count, fmt, dtype, a ring given, NULL
+ * scale_out, NULL x/out8 with n > 0), FP8_ERR_UNSUPPORTED (an fp32 job or one
+ * above FP8_QUANTIZE_SMALL_MAX), FP8_ERR_ALIGNMENT, FP8_ERR_CUDA. */
+#define FP8_QUANTIZE_SMALL_MAX 65536
+FP8LITE_API fp8_status fp8_quantize_current_many(const fp8_quantize_job* jobs, int32_t count, void* stream);
 
 /* Per-tensor-scaled FP8 GEMM with fused bias and bf16 output
  * [fp8.py@f4c44ebf, bullets on the fused bias and 3-D operands;

@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(fp8):
 
 
 def test_abi_version_and_status_strings(fp8):
-    assert fp8.fp8_abi_version() == 3
+    assert fp8.fp8_abi_version() == 4
     for code, name in [(0, "FP8_OK"), (1, "FP8_ERR_INVALID_ARG"), (2, "FP8_ERR_ALIGNMENT"),
                        (3, "FP8_ERR_UNSUPPORTED"), (4, "FP8_ERR_CUDA"), (5, "FP8_ERR_DEVICE_TIMEOUT")]:
         assert fp8.status_string(code) == name
@@ -124,6 +124,25 @@ def test_quantize_many_validation(fp8):
     assert status([(A, 64, 0, 3, S, A + 4096, None, S + 64)]) == fp8.FP8_ERR_INVALID_ARG     # bad dtype
     assert status([(A + 2, 64, 0, 0, S, A + 4096, None, S + 64)]) == fp8.FP8_ERR_ALIGNMENT
     assert fp8.raw_status("fp8_quantize_many", None, 1, None) == fp8.FP8_ERR_INVALID_ARG
+
+
+def test_quantize_current_many_validation(fp8):
+    def status(jobs, count=None):
+        arr = (fp8.fp8_quantize_job * max(len(jobs), 1))(*[fp8.fp8_quantize_job(*j) for j in jobs])
+        return fp8.raw_status("fp8_quantize_current_many", ctypes.cast(arr, ctypes.c_void_p),
+                              len(jobs) if count is None else count, None)
+    good = (A, 64, 0, 0, None, A + 4096, None, S + 64)   # x, n, fmt, dtype, ring, out8, amax_out, scale_out
+    assert status([good], count=0) == fp8.FP8_ERR_INVALID_ARG
+    assert status([good] * 9) == fp8.FP8_ERR_INVALID_ARG
+    assert status([(A, 64, 0, 0, S, A + 4096, None, S + 64)]) == fp8.FP8_ERR_INVALID_ARG      # a ring given
+    assert status([(A, 64, 0, 0, None, A + 4096, None, None)]) == fp8.FP8_ERR_INVALID_ARG    # no scale_out
+    assert status([(None, 64, 0, 0, None, A + 4096, None, S + 64)]) == fp8.FP8_ERR_INVALID_ARG  # no x
+    assert status([(A, 64, 2, 0, None, A + 4096, None, S + 64)]) == fp8.FP8_ERR_INVALID_ARG  # bad fmt
+    assert status([(A, 64, 0, 2, None, A + 4096, None, S + 64)]) == fp8.FP8_ERR_UNSUPPORTED  # fp32 input
+    assert status([(A, fp8.FP8_QUANTIZE_SMALL_MAX + 8, 0, 0, None, A + (1 << 20), None, S + 64)]) == \
+        fp8.FP8_ERR_UNSUPPORTED
+    assert status([(A + 8, 64, 0, 0, None, A + 4096, None, S + 64)]) == fp8.FP8_ERR_ALIGNMENT
+    assert status([(A, 64, 0, 0, None, A + 4096, S + 2, S + 64)]) == fp8.FP8_ERR_ALIGNMENT
 
 
 def test_mm_workspace_size_and_alignment(fp8):

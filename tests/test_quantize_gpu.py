@@ -93,6 +93,42 @@ def test_current_scaling_degenerate(g):
     assert np.array_equal(g.codes(q), want)
 
 
+def test_current_many_small_jobs(g):
+    """fp8_quantize_current_many: eight small tensors current-scaled in one
+    launch (bf16 and fp16, both formats, empty, ragged, all zeros, and every
+    bf16 bit pattern): each job's codes, amax and scale are the oracle's
+    current scaling, and equal fp8_quantize_ex on that tensor alone."""
+    import fp8_delayed_scaling_quantize_b200 as fp8
+    sizes = [65536, 0, 1, 7, 4097, 1000, 65535, 65536]
+    dtypes = [0, 1, 0, 1, 0, 0, 1, 0]
+    fmts = [E4M3, E5M2, E4M3, E4M3, E5M2, E4M3, E5M2, E5M2]
+    xs = []
+    for j, (n, dt) in enumerate(zip(sizes, dtypes)):
+        x = W.f32_normal((n,), 10.0 ** (j - 3), 5200 + j).to(torch.bfloat16 if dt == 0 else torch.float16)
+        xs.append(x)
+    xs[5] = torch.zeros(1000, dtype=torch.bfloat16)
+    xs[7] = W.bf16_bit_patterns()  # NaN and Inf included: amax = inf, so scale 1
+    xd = [x.cuda() if x.numel() else None for x in xs]
+    outs = [torch.empty(max(n, 1), dtype=torch.uint8, device="cuda") for n in sizes]
+    amaxs = [torch.full((1,), -1.0, device="cuda") for _ in sizes]
+    scales = [torch.full((1,), -1.0, device="cuda") for _ in sizes]
+    fp8.fp8_quantize_current_many([(xd[j], sizes[j], fmts[j], None, outs[j] if sizes[j] else None, amaxs[j],
+                                    scales[j], dtypes[j]) for j in range(len(sizes))])
+    for j, x in enumerate(xs):
+        n, what = sizes[j], f"job {j}"
+        want, a, sc = oracle.quantize_current(x.float().numpy(), fmts[j])
+        got = g.codes(outs[j])[:n]
+        nan = _nan_code(want, fmts[j])
+        assert np.array_equal(got[~nan], want[~nan]) and _nan_code(got[nan], fmts[j]).all(), what
+        assert g.f32(amaxs[j])[0] == a and g.f32(scales[j])[0] == sc, what
+        alone, a1, s1 = g.quantize_ex(x.cuda(), dtypes[j], fmts[j])
+        assert np.array_equal(g.codes(alone)[:n], got), what
+        assert g.f32(a1)[0] == g.f32(amaxs[j])[0] and g.f32(s1)[0] == g.f32(scales[j])[0], what
+    # amax_out is optional
+    fp8.fp8_quantize_current_many([(xd[0], sizes[0], fmts[0], None, outs[0], None, scales[0], dtypes[0])])
+    assert g.f32(scales[0])[0] == oracle.quantize_current(xs[0].float().numpy(), fmts[0])[2]
+
+
 def test_ring_hand_table_on_gpu(g):
     with open(os.path.join(GOLDEN, "ring_sequence.json")) as f:
         gold = json.load(f)
