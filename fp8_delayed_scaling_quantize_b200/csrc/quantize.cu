@@ -24,7 +24,11 @@
 //    next call (and for CUDA-graph replay) with no host involvement;
 //  * current: memset of the caller's amax word, an amax-only pass, then the
 //    quantize pass that derives the scale from that amax. For tensors that
-//    fit in L2 the second read is served from L2;
+//    fit in L2 the second read is served from L2. A bf16 / fp16 tensor of
+//    up to 65536 elements takes one launch instead: one 1024-thread block
+//    holds it in registers, reduces the amax, derives the scale and
+//    converts; up to 8 such tensors share one launch, a block each
+//    (fp8_quantize_current_many);
 //  * seeded delayed call: the current-scaling passes, then block 0 folds the
 //    measured amax into the ring (astrai/extension/fp8.py @4dc5e923, bullet
 //    on the _ScaleRing objects with their update and seed);
