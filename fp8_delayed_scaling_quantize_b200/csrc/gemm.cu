@@ -1131,7 +1131,11 @@ fp8_status launch(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, co
 // 128 x 128 k-block loads 32 KB for half the MMA work of a 128 x 256 one,
 // which loads 48 KB), and the wider tile costs less per output. Pairs of
 // 256 x 256 are used only with at least one such tile per SM (below that
-// their coarser grain loses). The pair's 256 x 128 tile (24 KB per SM per
+// their coarser grain loses) and at least 16 k-blocks: with 4 or 8 (K = 512,
+// 1024) each CTA's 128 x 256 epilogue outlasts its main loop and pairs lost
+// to one SM's 128 x 256 on every shape measured (4096^2 x 1024 18.9 against
+// 20.4 us, 64 x 512^3 16.2 against 19.3), while from 16 on they won
+// (4096^2 x 2048 28.5 against 31.0). The pair's 256 x 128 tile (24 KB per SM per
 // k-block) measured slower than one SM's 128 x 128 on the shapes it could
 // serve and is not chosen.
 //
@@ -1173,7 +1177,8 @@ inline TileChoice choose_tile(int64_t M, int64_t N, int64_t K, int64_t batch, bo
         const int64_t rounds = (tiles * split + units - 1) / units;
         return double(rounds) * double(kb_per) * t_k + t_epi;
     };
-    if (split == 1 && M > BM && N > 128 && tile_count(M, N, batch, true, 256) >= sms) return {true, 256, 1};
+    if (split == 1 && M > BM && N > 128 && kb >= 16 && tile_count(M, N, batch, true, 256) >= sms)
+        return {true, 256, 1};
     const bool pair_ok = M > BM;  // a pair's second CTA would hold only padding otherwise
     const TileChoice c[4] = {{false, 256, split}, {false, 128, split}, {false, 64, split}, {true, 256, split}};
     const double t[4] = {cost(false, 256, 0.48, 2.0), cost(false, 128, 0.40, 1.0),

@@ -196,21 +196,22 @@ def test_no_device_error_after_all(g):
 
 
 # ------------------------------------------- SM-pair (256-row) tile path ---
-# Shapes with at least one pair tile per SM (>= 148 tiles of 256 x 256) run
-# on SM pairs; compared in full, with ragged M (a last pair whose second CTA
-# lies wholly past M), ragged N and K, every layout, bias and batches.
+# Shapes with at least one pair tile per SM (>= 148 tiles of 256 x 256) and
+# at least 16 k-blocks run on SM pairs; compared in full, with ragged M (a
+# last pair whose second CTA lies wholly past M), ragged N and K, every
+# layout, bias and batches.
 
 @pytest.mark.parametrize("layout,M,N,K", [
-    (NT, 2400, 4096, 256), (NT, 2368, 4000, 160), (NN, 2560, 4096, 160),
-    (TN, 2560, 4096, 144), (TN, 2368, 4096, 128)])
+    (NT, 2400, 4096, 2048), (NT, 2368, 4000, 2032), (NN, 2560, 4096, 2032),
+    (TN, 2560, 4096, 2056), (TN, 2368, 4096, 2048)])
 def test_pair_tiles_full(g, layout, M, N, K):
     _full_check(g, layout, M, N, K, E4M3, E4M3, 1000 + M + N + K)
 
 
 @pytest.mark.parametrize("layout", [NT, NN, TN])
 def test_pair_tiles_bias_and_batches(g, layout):
-    _full_check(g, layout, 1280, 2560, 256, E5M2, E4M3, 1101, batch=3, bcast_b=True, pad_c=48, bias_kind=1)
-    _full_check(g, layout, 2560, 4096, 128, E4M3, E5M2, 1102, bias_kind=2)
+    _full_check(g, layout, 1280, 2560, 2048, E5M2, E4M3, 1101, batch=3, bcast_b=True, pad_c=48, bias_kind=1)
+    _full_check(g, layout, 2560, 4096, 2048, E4M3, E5M2, 1102, bias_kind=2)
 
 
 # Narrow NT problems with a long K (few output tiles, many k-blocks): ragged

@@ -102,7 +102,7 @@ def test_out8_layouts_formats_bias(g, case):
 def test_out8_pair_tiles(g):
     """Large enough for SM-pair tiles: each CTA of a pair folds its own amax
     and takes its own ticket."""
-    _run_case(g, NT, 2400, 4096, 256, E4M3, E4M3, E4M3, 3100)
+    _run_case(g, NT, 2400, 4096, 2048, E4M3, E4M3, E4M3, 3100)
 
 
 @pytest.mark.parametrize("layout", [NT, NN, TN])
