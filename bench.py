@@ -1042,12 +1042,25 @@ def oracle_sample_step(prep, frac=1, blk=1):
 
 
 def cpu_baseline_full_step():
-    """The oracle as it stands on one full step of the workload (rank 0)."""
+    """The oracle as it stands on one full step of the workload (rank 0), on
+    all the host's BLAS threads; beside it the same oracle held to one thread
+    on a 1/16 sample of the step."""
     prep = oracle_prepare(W.stack_tensors(0))
     dt, flops, elems = oracle_sample_step(prep)
-    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": _threads(), "kind": "oracle",
-            "sample": f"one full step: 12 delayed quantizes ({elems / 1e6:.1f} M elements) + 12 fp64 GEMMs "
-                      f"({flops / 1e9:.1f} GFLOP)", "seconds": round(dt, 2)}
+    out = {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": _threads(), "kind": "oracle",
+           "sample": f"one full step: 12 delayed quantizes ({elems / 1e6:.1f} M elements) + 12 fp64 GEMMs "
+                     f"({flops / 1e9:.1f} GFLOP)", "seconds": round(dt, 2)}
+    try:
+        from threadpoolctl import threadpool_limits
+    except ImportError:
+        return out
+    with threadpool_limits(limits=1):
+        dt1, f1, e1 = oracle_sample_step(prep, 16, 4)
+    out["single_thread"] = {"value": round(f1 / dt1 / 1e12, 6), "unit": "TFLOP/s", "cores": 1,
+                            "sample": f"1/16 of the step: the first 1/16 of each quantize input ({e1 / 1e6:.1f} M "
+                                      f"elements) and an (M/4) x (N/4) output block of each GEMM "
+                                      f"({f1 / 1e9:.1f} GFLOP)", "seconds": round(dt1, 2)}
+    return out
 
 
 REF_FRAC, REF_BLK = 256, 16
