@@ -1188,6 +1188,18 @@ inline TileChoice choose_tile(int64_t M, int64_t N, int64_t K, int64_t batch, bo
     double best_cost = 1e30;
     for (int i = 0; i < 4; ++i)
         if (t[i] < best_cost) { best = c[i]; best_cost = t[i]; }
+    // With at most 4 k-blocks a 128 x 256 tile's epilogue (about 2.1 us)
+    // outlasts its main loop while a 128 x 128 tile's (about 1.1 us) does not,
+    // so the rounds times the epilogue decide between the two widths. Measured
+    // on B200 over ten such shapes, this picks the faster of them in every case
+    // with a clear difference: 128 for 64 x 512^3 (15.1 us against 16.2) and
+    // 4096^2 x 512 (14.1 against 14.7), 256 for 2048^2 x 256 (5.4 against 5.6)
+    // and 4096 x 2048 x 128 (7.1 against 7.9), among others.
+    if (!best.pair && (best.bn == 256 || best.bn == 128) && split == 1 && kb <= 4) {
+        const int64_t r256 = (tile_count(M, N, batch, false, 256) + sms - 1) / sms;
+        const int64_t r128 = (tile_count(M, N, batch, false, 128) + sms - 1) / sms;
+        best = {false, double(r128) * 1.1 < double(r256) * 2.1 ? 128 : 256, 1};
+    }
     return best;
 }
 
@@ -1394,8 +1406,13 @@ fp8_status mm_impl(const uint8_t* a8, fp8_fmt fa, const uint8_t* b8, fp8_fmt fb,
     if (!o8.on && batch == 1 && split_k <= 1 && !swap_ab(M, N, layout)) {
         const TileChoice tc = choose_tile(M, N, K, 1, b_mn, sm_count(), split_k);
         const int64_t kb1 = (K + BK - 1) / BK;
-        if (!tc.pair && tc.bn == 256 && tc.split == 1 && choose_group_bn(&M, &N, &kb1, 1, sm_count()) == 256 &&
-            choose_narrow_tail(&M, &N, &kb1, 1, sm_count()) > 0) {
+        // only where it was measured to win: at least 8 k-blocks and at most
+        // two rounds of 256-wide tiles (NT 2048 x 3072 x 1024: 11.52 -> 11.01 us);
+        // with more rounds or fewer k-blocks the plain 128 x 256 launch was
+        // faster (4096^2 x 1024 18.9 against 21.6 us, 2048^2 x 256 5.4 against 5.6)
+        if (!tc.pair && tc.bn == 256 && tc.split == 1 && kb1 >= 8 &&
+            tile_count(M, N, 1, false, 256) <= 2 * int64_t(sm_count()) &&
+            choose_group_bn(&M, &N, &kb1, 1, sm_count()) == 256 && choose_narrow_tail(&M, &N, &kb1, 1, sm_count()) > 0) {
             const fp8_mm_problem one = {a8, b8, sa, sb, bias, bias_scale, out, M, N, K,
                                         int32_t(fa), int32_t(fb), int32_t(layout), int32_t(bias_fmt)};
             return mm_grouped_impl(&one, 1, stream);
